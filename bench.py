@@ -1,0 +1,446 @@
+#!/usr/bin/env python
+"""StateKV streaming-prefill benchmark: frames/s per layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload 8b_layer] [--l2 flush|resident]
+
+One step = one StateKV cache-builder step (attention, score pass, top-B select,
+gather + append) for one layer and one frame, in steady state (the compressed
+state is full).  Before the W untimed warm-up steps the stream is run through
+ceil(B/T) fill frames.  Inputs are seeded synthetic frames already resident in
+device memory.  Each timed step is bracketed by CUDA events on the launching
+stream; with --l2 flush (default) a 256 MiB buffer is written between steps,
+outside the events.  For N > 1 every rank runs an independent replica stream
+(no collective on the data path); value = all frames / max-over-ranks time.
+
+--impl reference times the float64 CPU oracle (rank 0 only) on the same
+workload: each step is one oracle step on a sample of the KV heads, scaled to
+the whole layer.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from kv_cache_selection_b200 import synthetic as Syn  # noqa: E402
+
+METRIC = "StateKV prefill frames/s per layer (8B shape, B=4096); % tensor-pipe peak"
+UNIT = "frames/s per layer"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ helpers --
+def rank_info():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
+            int(os.environ.get("WORLD_SIZE", 1)))
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def step_work(wl, m, S=1, causal=True):
+    """Algorithmic work of one step at C length m."""
+    T, Hq, Hkv, d = wl.T, wl.Hq, wl.Hkv, wl.d
+    esize = 2 if wl.dtype == "bf16" else 4
+    pairs = T * m + (T * (T + 1) // 2 if causal else T * T)   # visible (query, key) pairs per head
+    qk = 2 * S * Hq * d * pairs
+    m_new = min(wl.B, m + T)
+    L = m + T
+    gather_bytes = S * Hkv * (2 * 2 * m_new * d * esize + 2 * 8 * m_new) \
+        + S * Hkv * 2 * 2 * T * d * esize + S * T * 8
+    select_bytes = S * Hkv * L * 4 * 2 + S * Hkv * wl.B * 12
+    return {"attention": ("tensor", 2 * qk), "score": ("tensor", qk),
+            "select": ("hbm", select_bytes), "gather": ("hbm", gather_bytes)}
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            out_dir = os.path.join(ROOT, "gpurun_out") if os.path.isdir(os.path.join(ROOT, "gpurun_out")) \
+                else "/tmp"
+            self.path = os.path.join(out_dir, f"clocks_rank{self.gpu}_{os.getpid()}.csv")
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_stage, workload):
+    """Per-launch DRAM bytes from a committed ncu summary, if it is current."""
+    p = os.path.join(ROOT, "profiles", f"traffic_{kernel_stage}_{workload}.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+        if d.get("source_sha") != source_hash(d["sources"]):
+            return None
+        return float(d["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------------ our arm --
+def make_frames(wl, n_distinct, stream, dev):
+    fr = Syn.gen_frames(wl, n_distinct, stream=stream)
+    q = torch.stack([f[0] for f in fr]).to(dev)
+    k = torch.stack([f[1] for f in fr]).to(dev)
+    v = torch.stack([f[2] for f in fr]).to(dev)
+    return fr, q, k, v
+
+
+def run_ours(args, wl):
+    from kv_cache_selection_b200 import statekv as SKV
+
+    rank, local_rank, world = rank_info()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    K, W = args.steps, args.warmup
+    fill = math.ceil(wl.B / wl.T)
+    total_frames = fill + W + K
+    n_distinct = min(total_frames, args.distinct_frames)
+    fr_cpu, Q, Kf, Vf = make_frames(wl, n_distinct, rank, dev)
+    pos_all = torch.arange(total_frames * wl.T, dtype=torch.int32, device=dev).view(total_frames, wl.T)
+    out = torch.empty((wl.T, wl.Hq, wl.d), dtype=wl.torch_dtype, device=dev)
+    h = SKV.StateKV(wl.Hq, wl.Hkv, wl.d, wl.T, wl.B, max_frames=total_frames, dtype=wl.dtype)
+    h.reserve_layers(1)
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.int32, device=dev) if args.l2 == "flush" else None
+
+    def step(n):
+        i = n % n_distinct
+        h.prefill_frame(0, Q[i], Kf[i], Vf[i], pos_all[n], out)
+
+    for n in range(fill + W):
+        step(n)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    h.profile(True)
+    launches0 = h.kernel_launches()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    for j in range(K):
+        if flush is not None:
+            flush.fill_(j)
+        ev[j][0].record()
+        step(fill + W + j)
+        ev[j][1].record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    launches = h.kernel_launches() - launches0
+    stages = h.profile_read()
+    h.profile(False)
+    clk = clocks.stop()
+    ms_steps = [a.elapsed_time(b) for a, b in ev]
+    ms_total = sum(ms_steps)
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_total = float(t.item())
+
+    # ---- end to end through the host-buffer C-ABI call (pinned host memory)
+    e2e = None
+    if not args.no_e2e:
+        qh = torch.empty((wl.T, wl.Hq, wl.d), dtype=wl.torch_dtype).pin_memory()
+        kh = torch.empty((wl.T, wl.Hkv, wl.d), dtype=wl.torch_dtype).pin_memory()
+        vh = torch.empty_like(kh).pin_memory()
+        ph = torch.empty((wl.T,), dtype=torch.int32).pin_memory()
+        oh = torch.empty_like(qh).pin_memory()
+        he = SKV.StateKV(wl.Hq, wl.Hkv, wl.d, wl.T, wl.B, max_frames=total_frames, dtype=wl.dtype)
+        he.reserve_layers(1)
+        host_frames = [(f[0].contiguous().pin_memory(), f[1].contiguous().pin_memory(),
+                        f[2].contiguous().pin_memory()) for f in fr_cpu]
+
+        def host_step(n):
+            i = n % n_distinct
+            qh.copy_(host_frames[i][0])
+            kh.copy_(host_frames[i][1])
+            vh.copy_(host_frames[i][2])
+            ph.copy_(torch.arange(n * wl.T, (n + 1) * wl.T, dtype=torch.int32))
+            he.prefill_frame_host(0, qh, kh, vh, ph, oh)
+
+        for n in range(fill + W):
+            host_step(n)
+        torch.cuda.synchronize()
+        ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        for j in range(K):
+            if flush is not None:
+                flush.fill_(j)
+            torch.cuda.current_stream().synchronize()   # host buffers are refilled per step
+            n = fill + W + j
+            i = n % n_distinct
+            qh.copy_(host_frames[i][0])
+            kh.copy_(host_frames[i][1])
+            vh.copy_(host_frames[i][2])
+            ph.copy_(torch.arange(n * wl.T, (n + 1) * wl.T, dtype=torch.int32))
+            ev2[j][0].record()
+            he.prefill_frame_host(0, qh, kh, vh, ph, oh)
+            ev2[j][1].record()
+        torch.cuda.synchronize()
+        e2e_ms = sum(a.elapsed_time(b) for a, b in ev2)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        esize = 2 if wl.dtype == "bf16" else 4
+        h2d = (wl.T * wl.Hq * wl.d + 2 * wl.T * wl.Hkv * wl.d) * esize + wl.T * 4
+        d2h = wl.T * wl.Hq * wl.d * esize
+        e2e = {"value": world * K / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K,
+               "path": "statekv_prefill_frame_host (pinned host buffers, copies on the step's stream)"}
+        he.close()
+
+    if rank != 0:
+        h.close()
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    # ---- roofline of the dominant kernel
+    peaks, peak_src = load_peaks()
+    work = step_work(wl, wl.B)
+    stage_us = {k: (v[0] / max(v[1], 1)) * 1e3 for k, v in stages.items() if v[1]}
+    dominant = max(stage_us, key=lambda k: stages[k][0])
+    bound, amount = work.get(dominant, ("tensor", 0))
+    avg_s = stage_us[dominant] / 1e6
+    if bound == "tensor":
+        achieved = amount / avg_s / 1e12
+        peak = peaks["bf16_tflops"]
+        unit = "TFLOP/s"
+    else:
+        achieved = amount / avg_s / 1e9
+        peak = peaks["hbm_gbs"]
+        unit = "GB/s"
+    roofline = {"kernel": dominant, "bound": bound, "achieved": round(achieved, 2), "peak": peak,
+                "unit": unit, "frac": round(achieved / peak, 4),
+                "peak_source": f"{peak_src} ({'bf16 burst' if bound == 'tensor' else 'copy'})",
+                "algorithmic_per_launch": amount,
+                "traffic": ncu_traffic(dominant, wl.name)}
+    per_stage = {}
+    for k, us in stage_us.items():
+        b, amt = work.get(k, ("", 0))
+        if b == "tensor":
+            per_stage[k] = {"us": round(us, 2), "tflops": round(amt / us / 1e6, 1),
+                            "frac": round(amt / us / 1e6 / peaks["bf16_tflops"], 4)}
+        elif b == "hbm":
+            per_stage[k] = {"us": round(us, 2), "gbs": round(amt / us / 1e3, 1),
+                            "frac": round(amt / us / 1e3 / peaks["hbm_gbs"], 4)}
+        else:
+            per_stage[k] = {"us": round(us, 2)}
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, h, fr_cpu, fill + W + K, n_distinct, budget_s=args.cpu_budget)
+    h.close()
+
+    line = {
+        "metric": METRIC, "value": round(world * K / (ms_total / 1e3), 2), "unit": UNIT,
+        "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": round(ms_total / K, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+        "data": "synthetic",
+        "config": {"workload": f"{wl.name}: Hq={wl.Hq} Hkv={wl.Hkv} d={wl.d} T={wl.T} B={wl.B}, "
+                               f"steady state (C full), frame-causal, global select",
+                   "global_batch": world, "seq_len": wl.T, "frames_per_rank": total_frames,
+                   "l2": ("256 MiB buffer written between timed steps (outside the events)"
+                          if args.l2 == "flush" else "not flushed (C stays L2-resident across frames)"),
+                   "parallelism": f"replicas x{world} (no data-path collective)"},
+        "roofline": roofline,
+        "stages_us": per_stage,
+        "step_us_p50": round(statistics.median(ms_steps) * 1e3, 2),
+        "step_us_p99": round(sorted(ms_steps)[int(0.99 * (len(ms_steps) - 1))] * 1e3, 2),
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
+        "gpu_launches_per_step": launches / K, "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(wl, h, fr_cpu, n_next, n_distinct, budget_s=20.0, kv_heads=None):
+    """The oracle, as it stands, on a bounded sample of the same workload: steady
+    state steps from the GPU's own compressed state, on a subset of the KV heads
+    (each with its G query heads), scaled to the whole layer."""
+    from threadpoolctl import threadpool_info
+    from oracle import statekv_oracle as O
+
+    C = h.get_compressed(0)
+    m = C["len"]
+    G = wl.Hq // wl.Hkv
+    kvh = kv_heads or 1
+    st = O.LayerState.from_compressed(C["k"][0, :kvh, :m].cpu(), C["v"][0, :kvh, :m].cpu(),
+                                      C["pos"][0, :kvh, :m].cpu().numpy())
+    frames_done = 0
+    t0 = time.perf_counter()
+    n = n_next
+    while True:
+        q, k, v, _ = fr_cpu[n % n_distinct]
+        pos = torch.arange(n * wl.T, (n + 1) * wl.T).numpy()
+        st, _ = O.statekv_step(st, q[:, :kvh * G], k[:, :kvh], v[:, :kvh], pos, wl.B)
+        frames_done += 1
+        n += 1
+        el = time.perf_counter() - t0
+        if el > budget_s or frames_done >= 64:
+            break
+    threads = [p.get("num_threads", 1) for p in threadpool_info() if p.get("user_api") == "blas"]
+    frac = kvh / wl.Hkv
+    value = frames_done * frac / el
+    return {"value": round(value, 5), "unit": UNIT, "cores": int(max(threads) if threads else 1),
+            "host_cpus": os.cpu_count(), "kind": "oracle",
+            "sample": f"{frames_done} steady-state frames of {wl.name} on {kvh} of {wl.Hkv} KV heads "
+                      f"({kvh * G} query heads), float64 numpy oracle, {el:.1f} s; value scaled by "
+                      f"{wl.Hkv}/{kvh}"}
+
+
+# ------------------------------------------------------------ reference arm --
+def run_reference(args, wl):
+    rank, _, world = rank_info()
+    if rank != 0:
+        return
+    from threadpoolctl import threadpool_info
+    from oracle import statekv_oracle as O
+
+    K, W = args.steps, args.warmup
+    G = wl.Hq // wl.Hkv
+    # steady state needs a full C: build it from the oracle's own fill frames on
+    # one KV head group (this prologue is not timed)
+    kvh = 1
+    fill = math.ceil(wl.B / wl.T)
+    n_distinct = min(args.distinct_frames, fill + W + K, 32)
+    frames = Syn.gen_frames(wl, n_distinct)
+    st = O.LayerState.empty(kvh, wl.d)
+    for n in range(fill):
+        q, k, v, _ = frames[n % n_distinct]
+        pos = torch.arange(n * wl.T, (n + 1) * wl.T).numpy()
+        st, _ = O.statekv_step(st, q[:, :kvh * G], k[:, :kvh], v[:, :kvh], pos, wl.B)
+    t_steps = []
+    n = fill
+    for j in range(W + K):
+        q, k, v, _ = frames[n % n_distinct]
+        pos = torch.arange(n * wl.T, (n + 1) * wl.T).numpy()
+        t0 = time.perf_counter()
+        st, _ = O.statekv_step(st, q[:, :kvh * G], k[:, :kvh], v[:, :kvh], pos, wl.B)
+        dt = time.perf_counter() - t0
+        if j >= W:
+            t_steps.append(dt)
+        n += 1
+    frac = kvh / wl.Hkv
+    total = sum(t_steps) / frac        # scaled to all KV heads
+    value = K / total
+    threads = [p.get("num_threads", 1) for p in threadpool_info() if p.get("user_api") == "blas"]
+    cores = int(max(threads) if threads else 1)
+    sample = (f"each step: one float64 oracle step of {wl.name} in steady state on {kvh} of {wl.Hkv} "
+              f"KV heads ({kvh * G} query heads), time scaled by {wl.Hkv}/{kvh}")
+    line = {"metric": METRIC, "value": round(value, 5), "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": round(total / K * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": f"{wl.name}: Hq={wl.Hq} Hkv={wl.Hkv} d={wl.d} T={wl.T} B={wl.B}, "
+                                   f"steady state (C full), frame-causal, global select",
+                       "global_batch": 1, "seq_len": wl.T, "parallelism": "host cores"},
+            "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "host_cpus": os.cpu_count(), "sample": sample},
+            "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="8b_layer", choices=sorted(Syn.WORKLOADS))
+    ap.add_argument("--l2", choices=["flush", "resident"], default="flush")
+    ap.add_argument("--distinct-frames", type=int, default=96,
+                    help="distinct synthetic frames kept on the device (cycled)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle time")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = Syn.workload(args.workload)
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    main()

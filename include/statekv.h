@@ -1,0 +1,203 @@
+/*
+ * statekv.h — C ABI of the StateKV per-frame streaming-prefill library
+ * (libstatekv.so, sm_100a).
+ *
+ * Method: "Linear Scaling Video VLMs for Long Video Understanding" (StateKV).
+ * Citations name the summary page by title and the section on it:
+ *   P1  "线性扩展视频视觉语言模型用于长视频理解 Linear Scaling Video VLMs for Long
+ *       Video Understanding" (Chinese summary), section 方法步骤详情 (method steps).
+ *   P2  "Linear Scaling Video VLMs for Long Video Understanding" (section
+ *       summary), section 3.2 Method Overview, 3.3 Per-frame cache-builder
+ *       forward pass, Appendix A "Protocol", A.3 "Kernel considerations".
+ *   P3  "Technische Samenvatting: Lineair Schalende Video VLMs voor Lange Video
+ *       Begrip (StateKV)", section 2 "Architectuur en Mechanisme".
+ *
+ * Conventions for every call:
+ *   - Return 0 (STATEKV_OK) on success, a negative statekv_status on error.  On
+ *     error nothing is enqueued and the handle's state is unchanged;
+ *     statekv_last_error() holds a message.  No kernel traps on bad input: the
+ *     host validates first.
+ *   - "device pointer" arguments point to GPU global memory of the current
+ *     device, row-major and contiguous, with at least 16-byte alignment.  The
+ *     caller owns them; the library never frees or retains them past the call.
+ *   - "stream" is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls only enqueue work on it and never synchronise the host, except
+ *     where stated (allocation on first use of a layer).
+ *   - Shapes: S = n_streams (1 unless created batched), Hq query heads, Hkv KV
+ *     heads (Hq % Hkv == 0, query head h reads KV head h / (Hq/Hkv)), head
+ *     dimension d in {64, 128}, T tokens per frame, B the capacity of the
+ *     compressed state.
+ *   - Element type: STATEKV_BF16 (bfloat16, the graded path, tensor cores) or
+ *     STATEKV_F32 (float32, CUDA-core path).  Arithmetic is float32 in both.
+ */
+#ifndef STATEKV_H
+#define STATEKV_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct statekv_handle* statekv_t;
+
+typedef enum { STATEKV_BF16 = 0, STATEKV_F32 = 1 } statekv_dtype;
+
+/* Mask inside the current frame.  FRAME_CAUSAL (default): frame query i sees
+ * frame tokens t <= i (the backbone LLM is causal, P1 section 自注意力复杂度);
+ * FRAME_BIDIR: every frame token.  Entries of the compressed state are always
+ * visible. */
+typedef enum { STATEKV_MASK_FRAME_CAUSAL = 0, STATEKV_MASK_FRAME_BIDIR = 1 } statekv_mask;
+
+/* Selection granularity.  GLOBAL (default): one score per candidate summed over
+ * all query heads, one kept set per layer.  PER_KV_HEAD: scores summed over
+ * the query heads of each KV head, a kept set per KV head (P2 Appendix A
+ * "Protocol": sinks are kept per layer and KV head). */
+typedef enum { STATEKV_SELECT_GLOBAL = 0, STATEKV_SELECT_PER_KV_HEAD = 1 } statekv_select;
+
+typedef enum {
+  STATEKV_OK = 0,
+  STATEKV_ERR_INVALID_ARG = -1, /* null pointer, bad shape, bad enum          */
+  STATEKV_ERR_UNSUPPORTED = -2, /* d not in {64,128}, unsupported combination  */
+  STATEKV_ERR_CAPACITY = -3,    /* more frames than max_frames on a layer     */
+  STATEKV_ERR_OOM = -4,         /* device allocation failed                   */
+  STATEKV_ERR_CUDA = -5         /* a CUDA launch or runtime call failed       */
+} statekv_status;
+
+/* Create a handle for one video stream (S = 1).
+ * Allocates per-step scratch now; per-layer state (C and D) is allocated on a
+ * layer's first prefill_frame call (or by statekv_reserve_layers).
+ * max_frames bounds the frames per layer (D holds max_frames*T tokens).
+ * B >= 0 (B = 0: no cross-frame context).  Errors: INVALID_ARG, UNSUPPORTED,
+ * OOM, CUDA.  *h is set only on success. */
+int statekv_create(statekv_t* h, int Hq, int Hkv, int d, int T, int B, int max_frames,
+                   int dtype, int mask_mode, int select_mode);
+
+/* Same as statekv_create for n_streams independent video streams processed
+ * together: every tensor below gains a leading [S] dimension and each stream
+ * keeps its own C and D.  All streams advance one frame per call. */
+int statekv_create_batched(statekv_t* h, int n_streams, int Hq, int Hkv, int d, int T,
+                           int B, int max_frames, int dtype, int mask_mode,
+                           int select_mode);
+
+/* Allocate the state of layers 0..n_layers-1 now (synchronous; device memory
+ * zero-filled).  Call before capturing prefill calls in a CUDA graph. */
+int statekv_reserve_layers(statekv_t h, int n_layers);
+
+/* One StateKV cache-builder step for one layer and the next frame
+ * (P1 section 方法步骤详情; P2 section 3.3; P3 section 2 "Het Proces"):
+ *   1. out = softmax(q [C_{n-1}; k]^T / sqrt(d)) [C_{n-1}; v]  (mask_mode);
+ *   2. D <- D || (k, v, pos);
+ *   3. score_j = sum over the frame's queries i (and heads) of P_ij for every
+ *      candidate j of the pool C_{n-1} followed by the frame's tokens;
+ *   4. C_n = the B best candidates by (score desc, position asc), stored in
+ *      ascending position order (all candidates while m + T <= B).
+ * Inputs (device pointers, element type = dtype):
+ *   q   [S][T][Hq][d]   queries, RoPE already applied at absolute positions
+ *   k,v [S][T][Hkv][d]  keys (RoPE applied) and values
+ *   pos [S][T] int32    absolute ("virtual") positions (P2 section 3.3); they
+ *                       must increase along the stream: every frame's positions
+ *                       ascending and above all earlier frames' positions.
+ *                       The library stores them and never re-rotates.
+ * Output (device pointer): out [S][T][Hq][d] (dtype).
+ * Frame n of a layer must follow frame n-1 of that layer on the same stream
+ * order; layers may interleave.  Errors: INVALID_ARG, CAPACITY, OOM (first use
+ * of a layer), CUDA. */
+int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k,
+                          const void* v, const int32_t* pos, void* out, void* stream);
+
+/* statekv_prefill_frame with HOST buffers: q, k, v, pos are read from and out
+ * is written to host memory (same layouts; page-locked memory makes the copies
+ * asynchronous, pageable memory is accepted).  The call enqueues the
+ * host-to-device copies into library-owned staging buffers, the step, and the
+ * device-to-host copy of out on `stream`; out is complete once the stream has
+ * reached that point (synchronise the stream before reading it).  Calls on one
+ * handle reuse the same staging buffers, so successive host calls are ordered
+ * by the stream.  Errors: as statekv_prefill_frame. */
+int statekv_prefill_frame_host(statekv_t h, int layer, const void* q, const void* k,
+                               const void* v, const int32_t* pos, void* out, void* stream);
+
+/* Borrow the compressed state C_n of a layer (device pointers owned by the
+ * library; valid until the next prefill_frame on that layer or destroy):
+ *   k,v   [S][Hkv][B][d] (dtype), rows [0, len) valid, ascending position
+ *   pos   [S][Hkv][B] int32, score [S][Hkv][B] float32 (the score each kept
+ *         entry earned in the frame that selected it).  In GLOBAL mode the Hkv
+ *         rows of pos/score are identical.
+ *   len   current length m = min(B, frames*T).
+ * Any output pointer may be NULL.  Errors: INVALID_ARG (unknown layer). */
+int statekv_get_compressed(statekv_t h, int layer, const void** k, const void** v,
+                           const int32_t** pos, const float** score, int* len);
+
+/* Borrow the detailed state D of a layer (P2 section 3.2: every frame token,
+ * kept for decoding):
+ *   k,v [S][Hkv][max_frames*T][d] (dtype), tokens [0, len) valid, in arrival
+ *   order; pos [S][max_frames*T] int32.  len = frames*T.
+ * Valid until destroy.  Errors: INVALID_ARG. */
+int statekv_get_detailed(statekv_t h, int layer, const void** k, const void** v,
+                         const int32_t** pos, int* len);
+
+/* Borrow the per-row statistics of the most recent prefill_frame (any layer):
+ *   lse        [S][Hq][T] float32, natural-log log-sum-exp of each query row;
+ *   pool_score [S][Hkv][B+T] float32, the score of every pool candidate
+ *              (C entries first, then frame tokens; rows identical in GLOBAL
+ *              mode); entries [0, pool_len) valid.
+ * Valid until the next prefill_frame.  Any output pointer may be NULL. */
+int statekv_get_step_stats(statekv_t h, const float** lse, const float** pool_score,
+                           int* pool_len);
+
+/* Kernel stages of one step, for statekv_profile_read. */
+typedef enum {
+  STATEKV_STAGE_ATTENTION = 0,         /* (a) attention main kernel            */
+  STATEKV_STAGE_ATTENTION_COMBINE = 1, /* (a) merge of key-split partials      */
+  STATEKV_STAGE_SCORE = 2,             /* (b) score pass                       */
+  STATEKV_STAGE_SELECT = 3,            /* (c) top-B select                     */
+  STATEKV_STAGE_GATHER = 4,            /* (d) gather into C_n + append to D    */
+  STATEKV_N_STAGES = 8
+} statekv_stage;
+
+/* Per-stage device timing: when on, every later prefill_frame records a CUDA
+ * event pair around each kernel on the call's stream (a few microseconds of
+ * extra enqueue cost; leave off in production).  Turning it off drops
+ * unread records. */
+int statekv_profile_enable(statekv_t h, int on);
+
+/* Accumulated device time and launch count per stage since the last read:
+ * ms[STATEKV_N_STAGES] milliseconds, launches[STATEKV_N_STAGES] (either may be
+ * NULL).  Waits for the recorded events (host synchronisation), then resets. */
+int statekv_profile_read(statekv_t h, double* ms, long long* launches);
+
+/* Number of kernels this handle has launched since it was created. */
+long long statekv_kernel_launches(statekv_t h);
+
+/* Frames processed so far on a layer (0 for a layer never called). */
+int statekv_frames(statekv_t h, int layer);
+
+/* Release all device memory of the handle (synchronises the device first). */
+int statekv_destroy(statekv_t h);
+
+/* Message of the handle's last error ("" if none); h may be NULL for errors of
+ * calls that had no handle (create, full_causal_prefill). */
+const char* statekv_last_error(statekv_t h);
+
+/* Full causal self-attention over n_tokens tokens: the quadratic comparator
+ * (P2 section 4 "Compute scaling"; P2 A.3: the full-attention baseline).
+ *   q [n_tokens][Hq][d], k,v [n_tokens][Hkv][d] (device, dtype);
+ *   out [n_tokens][Hq][d] (device, dtype);
+ *   lse [Hq][n_tokens] float32 natural-log (device) or NULL.
+ * Token i attends to tokens 0..i.  Scratch is allocated by the library on
+ * first use and kept (grown as needed) until process exit.
+ * Errors: INVALID_ARG, UNSUPPORTED, OOM, CUDA. */
+int full_causal_prefill(const void* q, const void* k, const void* v, int n_tokens, int Hq,
+                        int Hkv, int d, int dtype, void* out, float* lse, void* stream);
+
+/* full_causal_prefill over n_seq independent sequences of n_tokens each:
+ * every tensor gains a leading [n_seq] dimension (lse: [n_seq][Hq][n_tokens]). */
+int full_causal_prefill_batched(const void* q, const void* k, const void* v, int n_seq,
+                                int n_tokens, int Hq, int Hkv, int d, int dtype, void* out,
+                                float* lse, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STATEKV_H */

@@ -1,0 +1,102 @@
+// Shared device helpers and kernel argument blocks of libstatekv (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace skv {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T>
+__device__ __forceinline__ T from_f(float x);
+template <>
+__device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Attention of a block of query rows over a two-segment key pool:
+//   segment A = compressed state rows j < m (always visible),
+//   segment B = the frame's (or sequence's) tokens t < nb; with `causal`,
+//   query row i sees t <= i.
+// Element strides; every tensor is indexed [s] first.
+struct AttnArgs {
+  const void* q;       // q[s][i][h][dd]
+  long long q_s;       // stride of s
+  int q_row;           // stride of i (= Hq*d)
+  const void* ka;      // ka[s][g][j][dd]
+  const void* va;
+  long long a_s, a_g;  // strides of s and g (row stride = d)
+  int m;
+  const void* kb;      // kb[s][t][g][dd]
+  const void* vb;
+  long long b_s;
+  int b_row;           // stride of t (= Hkv*d)
+  int nb;
+  void* out;           // out[s][i][h][dd], same strides as q
+  float* lse;          // lse[s][h][i] natural log, may be null
+  long long lse_s;     // stride of s (= Hq*n_rows)
+  int n_rows;          // query rows per head
+  int Hq, Hkv;
+  int causal;
+  float scale_log2;    // log2(e)/sqrt(d)
+};
+
+// Column mass of the normalised softmax weights over one KV group's query
+// heads: part[s][g][j] = sum_{h in g} sum_i exp(s_hij - lse_hi).
+struct ScoreArgs {
+  const void* q;
+  long long q_s;
+  int q_row;
+  const void* ka;
+  long long a_s, a_g;
+  int m;
+  const void* kb;
+  long long b_s;
+  int b_row;
+  int nb;
+  const float* lse;    // lse[s][h][i] natural log
+  long long lse_s;
+  float* part;         // part[s][g][j]
+  long long part_s;
+  int part_g;
+  int n_rows, Hq, Hkv, causal;
+  float scale_log2;
+};
+
+// Top-B selection over the pool of one (stream, selection group).
+struct SelectArgs {
+  const float* part;      // part[s][g][j], j < m + T
+  long long part_s;
+  int part_g;
+  float* pool_score;      // out, same layout as part
+  const int32_t* pos_c;   // current C positions [s][g][B]
+  const int32_t* pos_f;   // frame positions [s][T]
+  int32_t* idx;           // out [s][g][B] kept pool indices, ascending
+  int32_t* pos_new;       // out [s][g][B]
+  float* score_new;       // out [s][g][B]
+  int Hkv, m, T, B, global;
+};
+
+// Gather of the kept rows into the next C buffer plus the append of the
+// frame's K/V to D.
+struct GatherArgs {
+  const void* kc;  const void* vc;   // current C [s][g][B][d]
+  const void* kf;  const void* vf;   // frame [s][t][g][d]
+  void* kc_new;    void* vc_new;     // next C [s][g][B][d]
+  const int32_t* idx;                // [s][g][B]
+  void* kd;        void* vd;         // D [s][g][max_tok][d]
+  int32_t* pos_d;                    // [s][max_tok]
+  const int32_t* pos_f;              // [s][T]
+  int Hkv, T, B, m, m_new, row_bytes, global, d_len, max_tok;
+  int S;
+};
+
+}  // namespace skv

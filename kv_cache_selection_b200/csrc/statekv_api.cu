@@ -1,0 +1,564 @@
+// Host side of libstatekv: the C ABI declared in include/statekv.h, per-layer
+// state (compressed C, detailed D) and the launch sequence of one step.
+//
+// One StateKV step ("Linear Scaling Video VLMs for Long Video Understanding",
+// P1 section 方法步骤详情; P2 section 3.3) is enqueued as
+//   (a) attention of the frame's queries over [C_{n-1}; frame]  -> out, lse
+//   (b) score pass: column mass of the normalised weights       -> partials
+//   (c) top-B select over the pool                              -> kept list
+//   (d) gather of the kept rows into the other C buffer + append to D
+// on the caller's stream with no host synchronisation.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "../../include/statekv.h"
+#include "kernels.h"
+
+namespace {
+
+thread_local std::string g_free_error;  // errors of calls without a handle
+
+struct LayerState {
+  bool ready = false;
+  int frames = 0;
+  int m = 0;    // current C length
+  int cur = 0;  // index of the current C buffer
+  void* kc[2] = {nullptr, nullptr};
+  void* vc[2] = {nullptr, nullptr};
+  int32_t* posc[2] = {nullptr, nullptr};
+  float* scorec[2] = {nullptr, nullptr};
+  void* kd = nullptr;
+  void* vd = nullptr;
+  int32_t* posd = nullptr;
+};
+
+}  // namespace
+
+struct statekv_handle {
+  int S = 1, Hq = 0, Hkv = 0, d = 0, T = 0, B = 0, max_frames = 0;
+  int dtype = 0, mask = 0, select = 0;
+  int n_sm = 148;
+  int device = 0;
+  size_t esize = 2;
+  std::vector<LayerState> layers;
+  // per-step scratch
+  float* lse = nullptr;         // [S][Hq][T]
+  float* part = nullptr;        // [S][Hkv][B+T]
+  float* pool_score = nullptr;  // [S][Hkv][B+T]
+  int32_t* idx = nullptr;       // [S][Hkv][max(B,1)]
+  // staging for statekv_prefill_frame_host (allocated on first use)
+  void* stage_q = nullptr;
+  void* stage_k = nullptr;
+  void* stage_v = nullptr;
+  void* stage_out = nullptr;
+  int32_t* stage_pos = nullptr;
+  int last_pool_len = 0;
+  std::string err;
+  std::vector<void*> allocs;
+  // launch accounting and optional per-stage event timing
+  long long launches = 0;
+  bool prof = false;
+  struct Rec {
+    int stage;
+    cudaEvent_t a, b;
+  };
+  std::vector<Rec> recs;
+  std::vector<cudaEvent_t> ev_free;
+};
+
+namespace {
+
+int set_err(statekv_t h, int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  if (h) h->err = buf;
+  else g_free_error = buf;
+  return code;
+}
+
+int dev_alloc(statekv_t h, void** p, size_t bytes) {
+  bytes = std::max<size_t>(bytes, 16);
+  cudaError_t e = cudaMalloc(p, bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    *p = nullptr;
+    return set_err(h, STATEKV_ERR_OOM, "cudaMalloc(%zu) failed: %s", bytes, cudaGetErrorString(e));
+  }
+  e = cudaMemset(*p, 0, bytes);
+  if (e != cudaSuccess) {
+    cudaFree(*p);
+    *p = nullptr;
+    return set_err(h, STATEKV_ERR_CUDA, "cudaMemset failed: %s", cudaGetErrorString(e));
+  }
+  h->allocs.push_back(*p);
+  return STATEKV_OK;
+}
+
+int check_shape(statekv_t h, int S, int Hq, int Hkv, int d, int T, int B, int max_frames, int dtype,
+                int mask, int select) {
+  if (S < 1 || Hq < 1 || Hkv < 1 || T < 1 || B < 0 || max_frames < 1)
+    return set_err(h, STATEKV_ERR_INVALID_ARG,
+                   "bad shape: S=%d Hq=%d Hkv=%d T=%d B=%d max_frames=%d", S, Hq, Hkv, T, B,
+                   max_frames);
+  if (Hq % Hkv != 0) return set_err(h, STATEKV_ERR_INVALID_ARG, "Hq (%d) %% Hkv (%d) != 0", Hq, Hkv);
+  if (dtype != STATEKV_BF16 && dtype != STATEKV_F32)
+    return set_err(h, STATEKV_ERR_INVALID_ARG, "bad dtype %d", dtype);
+  if (mask != STATEKV_MASK_FRAME_CAUSAL && mask != STATEKV_MASK_FRAME_BIDIR)
+    return set_err(h, STATEKV_ERR_INVALID_ARG, "bad mask_mode %d", mask);
+  if (select != STATEKV_SELECT_GLOBAL && select != STATEKV_SELECT_PER_KV_HEAD)
+    return set_err(h, STATEKV_ERR_INVALID_ARG, "bad select_mode %d", select);
+  if (d != 64 && d != 128) return set_err(h, STATEKV_ERR_UNSUPPORTED, "head dim %d not in {64,128}", d);
+  if ((long long)B + T > 49152)
+    return set_err(h, STATEKV_ERR_UNSUPPORTED, "pool B+T=%lld above 49152", (long long)B + T);
+  if ((long long)max_frames * T > (1LL << 30))
+    return set_err(h, STATEKV_ERR_UNSUPPORTED, "max_frames*T too large");
+  return STATEKV_OK;
+}
+
+int alloc_layer(statekv_t h, LayerState& L) {
+  const size_t cbytes = (size_t)h->S * h->Hkv * h->B * h->d * h->esize;
+  const size_t cint = (size_t)h->S * h->Hkv * h->B * 4;
+  const size_t max_tok = (size_t)h->max_frames * h->T;
+  const size_t dbytes = (size_t)h->S * h->Hkv * max_tok * h->d * h->esize;
+  int rc;
+  for (int b = 0; b < 2; ++b) {
+    if ((rc = dev_alloc(h, &L.kc[b], cbytes))) return rc;
+    if ((rc = dev_alloc(h, &L.vc[b], cbytes))) return rc;
+    if ((rc = dev_alloc(h, (void**)&L.posc[b], cint))) return rc;
+    if ((rc = dev_alloc(h, (void**)&L.scorec[b], cint))) return rc;
+  }
+  if ((rc = dev_alloc(h, &L.kd, dbytes))) return rc;
+  if ((rc = dev_alloc(h, &L.vd, dbytes))) return rc;
+  if ((rc = dev_alloc(h, (void**)&L.posd, (size_t)h->S * max_tok * 4))) return rc;
+  L.ready = true;
+  return STATEKV_OK;
+}
+
+int get_layer(statekv_t h, int layer, LayerState** out) {
+  if (layer < 0) return set_err(h, STATEKV_ERR_INVALID_ARG, "negative layer %d", layer);
+  if ((size_t)layer >= h->layers.size()) h->layers.resize(layer + 1);
+  LayerState& L = h->layers[layer];
+  if (!L.ready) {
+    int rc = alloc_layer(h, L);
+    if (rc) return rc;
+  }
+  *out = &L;
+  return STATEKV_OK;
+}
+
+cudaEvent_t take_event(statekv_t h) {
+  if (!h->ev_free.empty()) {
+    cudaEvent_t e = h->ev_free.back();
+    h->ev_free.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return e;
+}
+
+// Brackets one kernel launch: counts it and, when profiling, records an event
+// pair on the launch stream.
+struct StageScope {
+  statekv_t h;
+  cudaStream_t st;
+  int stage;
+  cudaEvent_t a = nullptr;
+  StageScope(statekv_t h_, cudaStream_t st_, int stage_) : h(h_), st(st_), stage(stage_) {
+    if (h->prof && (a = take_event(h)) != nullptr) cudaEventRecord(a, st);
+  }
+  void done() {
+    ++h->launches;
+    if (!a) return;
+    cudaEvent_t b = take_event(h);
+    if (!b) {
+      h->ev_free.push_back(a);
+      return;
+    }
+    cudaEventRecord(b, st);
+    h->recs.push_back({stage, a, b});
+  }
+};
+
+int launch_err(statekv_t h, cudaError_t e, const char* what) {
+  return set_err(h, STATEKV_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString(e));
+}
+
+}  // namespace
+
+extern "C" {
+
+int statekv_create_batched(statekv_t* out, int n_streams, int Hq, int Hkv, int d, int T, int B,
+                           int max_frames, int dtype, int mask_mode, int select_mode) {
+  if (!out) return set_err(nullptr, STATEKV_ERR_INVALID_ARG, "null handle pointer");
+  int rc = check_shape(nullptr, n_streams, Hq, Hkv, d, T, B, max_frames, dtype, mask_mode, select_mode);
+  if (rc) return rc;
+  statekv_t h = new (std::nothrow) statekv_handle();
+  if (!h) return set_err(nullptr, STATEKV_ERR_OOM, "host allocation failed");
+  h->S = n_streams;
+  h->Hq = Hq;
+  h->Hkv = Hkv;
+  h->d = d;
+  h->T = T;
+  h->B = B;
+  h->max_frames = max_frames;
+  h->dtype = dtype;
+  h->mask = mask_mode;
+  h->select = select_mode;
+  h->esize = dtype == STATEKV_BF16 ? 2 : 4;
+  cudaError_t e = cudaGetDevice(&h->device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&h->n_sm, cudaDevAttrMultiProcessorCount, h->device);
+  if (e != cudaSuccess) {
+    set_err(nullptr, STATEKV_ERR_CUDA, "no CUDA device: %s", cudaGetErrorString(e));
+    delete h;
+    return STATEKV_ERR_CUDA;
+  }
+  const size_t pool = (size_t)B + T;
+  if ((rc = dev_alloc(h, (void**)&h->lse, (size_t)n_streams * Hq * T * 4)) ||
+      (rc = dev_alloc(h, (void**)&h->part, (size_t)n_streams * Hkv * pool * 4)) ||
+      (rc = dev_alloc(h, (void**)&h->pool_score, (size_t)n_streams * Hkv * pool * 4)) ||
+      (rc = dev_alloc(h, (void**)&h->idx, (size_t)n_streams * Hkv * std::max(B, 1) * 4))) {
+    g_free_error = h->err;
+    statekv_destroy(h);
+    return rc;
+  }
+  *out = h;
+  return STATEKV_OK;
+}
+
+int statekv_create(statekv_t* out, int Hq, int Hkv, int d, int T, int B, int max_frames, int dtype,
+                   int mask_mode, int select_mode) {
+  return statekv_create_batched(out, 1, Hq, Hkv, d, T, B, max_frames, dtype, mask_mode, select_mode);
+}
+
+int statekv_reserve_layers(statekv_t h, int n_layers) {
+  if (!h) return set_err(nullptr, STATEKV_ERR_INVALID_ARG, "null handle");
+  if (n_layers < 0) return set_err(h, STATEKV_ERR_INVALID_ARG, "negative layer count");
+  for (int l = 0; l < n_layers; ++l) {
+    LayerState* L;
+    int rc = get_layer(h, l, &L);
+    if (rc) return rc;
+  }
+  return STATEKV_OK;
+}
+
+int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, const void* v,
+                          const int32_t* pos, void* out, void* stream) {
+  if (!h) return set_err(nullptr, STATEKV_ERR_INVALID_ARG, "null handle");
+  if (!q || !k || !v || !pos || !out)
+    return set_err(h, STATEKV_ERR_INVALID_ARG, "null input/output pointer");
+  if (((uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)out) & 15)
+    return set_err(h, STATEKV_ERR_INVALID_ARG, "q/k/v/out must be 16-byte aligned");
+  if (layer >= 0 && (size_t)layer < h->layers.size() && h->layers[layer].ready &&
+      h->layers[layer].frames >= h->max_frames)
+    return set_err(h, STATEKV_ERR_CAPACITY, "layer %d already holds max_frames=%d frames", layer,
+                   h->max_frames);
+  LayerState* L;
+  int rc = get_layer(h, layer, &L);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int S = h->S, Hq = h->Hq, Hkv = h->Hkv, d = h->d, T = h->T, B = h->B;
+  const int m = L->m, cur = L->cur, nxt = cur ^ 1;
+  const int pool = B + T;
+  const int m_new = std::min(B, m + T);
+  const float scale_log2 = skv::kLog2e / sqrtf((float)d);
+  cudaError_t e;
+
+  // (a) attention over [C_{n-1}; frame]
+  skv::AttnArgs aa{};
+  aa.q = q;
+  aa.q_s = (long long)T * Hq * d;
+  aa.q_row = Hq * d;
+  aa.ka = L->kc[cur];
+  aa.va = L->vc[cur];
+  aa.a_s = (long long)Hkv * B * d;
+  aa.a_g = (long long)B * d;
+  aa.m = m;
+  aa.kb = k;
+  aa.vb = v;
+  aa.b_s = (long long)T * Hkv * d;
+  aa.b_row = Hkv * d;
+  aa.nb = T;
+  aa.out = out;
+  aa.lse = h->lse;
+  aa.lse_s = (long long)Hq * T;
+  aa.n_rows = T;
+  aa.Hq = Hq;
+  aa.Hkv = Hkv;
+  aa.causal = h->mask == STATEKV_MASK_FRAME_CAUSAL;
+  aa.scale_log2 = scale_log2;
+  {
+    StageScope sc(h, st, STATEKV_STAGE_ATTENTION);
+    if ((e = skv::launch_attn_simt(aa, h->dtype, d, S, st)) != cudaSuccess) return launch_err(h, e, "attention");
+    sc.done();
+  }
+
+  // (b) score pass
+  skv::ScoreArgs sa{};
+  sa.q = q;
+  sa.q_s = aa.q_s;
+  sa.q_row = aa.q_row;
+  sa.ka = aa.ka;
+  sa.a_s = aa.a_s;
+  sa.a_g = aa.a_g;
+  sa.m = m;
+  sa.kb = k;
+  sa.b_s = aa.b_s;
+  sa.b_row = aa.b_row;
+  sa.nb = T;
+  sa.lse = h->lse;
+  sa.lse_s = aa.lse_s;
+  sa.part = h->part;
+  sa.part_s = (long long)Hkv * pool;
+  sa.part_g = pool;
+  sa.n_rows = T;
+  sa.Hq = Hq;
+  sa.Hkv = Hkv;
+  sa.causal = aa.causal;
+  sa.scale_log2 = scale_log2;
+  {
+    StageScope sc(h, st, STATEKV_STAGE_SCORE);
+    if ((e = skv::launch_score_simt(sa, h->dtype, d, S, st)) != cudaSuccess) return launch_err(h, e, "score");
+    sc.done();
+  }
+
+  // (c) top-B select
+  skv::SelectArgs se{};
+  se.part = h->part;
+  se.part_s = sa.part_s;
+  se.part_g = pool;
+  se.pool_score = h->pool_score;
+  se.pos_c = L->posc[cur];
+  se.pos_f = pos;
+  se.idx = h->idx;
+  se.pos_new = L->posc[nxt];
+  se.score_new = L->scorec[nxt];
+  se.Hkv = Hkv;
+  se.m = m;
+  se.T = T;
+  se.B = B;
+  se.global = h->select == STATEKV_SELECT_GLOBAL;
+  {
+    StageScope sc(h, st, STATEKV_STAGE_SELECT);
+    if ((e = skv::launch_select(se, S, st)) != cudaSuccess) return launch_err(h, e, "select");
+    sc.done();
+  }
+
+  // (d) gather into C_n + append to D
+  skv::GatherArgs ga{};
+  ga.kc = L->kc[cur];
+  ga.vc = L->vc[cur];
+  ga.kf = k;
+  ga.vf = v;
+  ga.kc_new = L->kc[nxt];
+  ga.vc_new = L->vc[nxt];
+  ga.idx = h->idx;
+  ga.kd = L->kd;
+  ga.vd = L->vd;
+  ga.pos_d = L->posd;
+  ga.pos_f = pos;
+  ga.Hkv = Hkv;
+  ga.T = T;
+  ga.B = B;
+  ga.m = m;
+  ga.m_new = m_new;
+  ga.row_bytes = (int)(d * h->esize);
+  ga.global = se.global;
+  ga.d_len = L->frames * T;
+  ga.max_tok = h->max_frames * T;
+  ga.S = S;
+  {
+    StageScope sc(h, st, STATEKV_STAGE_GATHER);
+    if ((e = skv::launch_gather(ga, h->n_sm, st)) != cudaSuccess) return launch_err(h, e, "gather");
+    sc.done();
+  }
+
+  L->m = m_new;
+  L->cur = nxt;
+  L->frames += 1;
+  h->last_pool_len = m + T;
+  return STATEKV_OK;
+}
+
+int statekv_prefill_frame_host(statekv_t h, int layer, const void* q, const void* k, const void* v,
+                               const int32_t* pos, void* out, void* stream) {
+  if (!h) return set_err(nullptr, STATEKV_ERR_INVALID_ARG, "null handle");
+  if (!q || !k || !v || !pos || !out)
+    return set_err(h, STATEKV_ERR_INVALID_ARG, "null input/output pointer");
+  const size_t qb = (size_t)h->S * h->T * h->Hq * h->d * h->esize;
+  const size_t kb = (size_t)h->S * h->T * h->Hkv * h->d * h->esize;
+  const size_t pb = (size_t)h->S * h->T * 4;
+  int rc;
+  if (!h->stage_q) {
+    if ((rc = dev_alloc(h, &h->stage_q, qb)) || (rc = dev_alloc(h, &h->stage_k, kb)) ||
+        (rc = dev_alloc(h, &h->stage_v, kb)) || (rc = dev_alloc(h, &h->stage_out, qb)) ||
+        (rc = dev_alloc(h, (void**)&h->stage_pos, pb)))
+      return rc;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if ((e = cudaMemcpyAsync(h->stage_q, q, qb, cudaMemcpyHostToDevice, st)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(h->stage_k, k, kb, cudaMemcpyHostToDevice, st)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(h->stage_v, v, kb, cudaMemcpyHostToDevice, st)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(h->stage_pos, pos, pb, cudaMemcpyHostToDevice, st)) != cudaSuccess)
+    return set_err(h, STATEKV_ERR_CUDA, "host-to-device copy failed: %s", cudaGetErrorString(e));
+  rc = statekv_prefill_frame(h, layer, h->stage_q, h->stage_k, h->stage_v, h->stage_pos, h->stage_out,
+                             stream);
+  if (rc) return rc;
+  if ((e = cudaMemcpyAsync(out, h->stage_out, qb, cudaMemcpyDeviceToHost, st)) != cudaSuccess)
+    return set_err(h, STATEKV_ERR_CUDA, "device-to-host copy failed: %s", cudaGetErrorString(e));
+  return STATEKV_OK;
+}
+
+int statekv_get_compressed(statekv_t h, int layer, const void** k, const void** v, const int32_t** pos,
+                           const float** score, int* len) {
+  if (!h) return set_err(nullptr, STATEKV_ERR_INVALID_ARG, "null handle");
+  if (layer < 0 || (size_t)layer >= h->layers.size() || !h->layers[layer].ready)
+    return set_err(h, STATEKV_ERR_INVALID_ARG, "unknown layer %d", layer);
+  const LayerState& L = h->layers[layer];
+  if (k) *k = L.kc[L.cur];
+  if (v) *v = L.vc[L.cur];
+  if (pos) *pos = L.posc[L.cur];
+  if (score) *score = L.scorec[L.cur];
+  if (len) *len = L.m;
+  return STATEKV_OK;
+}
+
+int statekv_get_detailed(statekv_t h, int layer, const void** k, const void** v, const int32_t** pos,
+                         int* len) {
+  if (!h) return set_err(nullptr, STATEKV_ERR_INVALID_ARG, "null handle");
+  if (layer < 0 || (size_t)layer >= h->layers.size() || !h->layers[layer].ready)
+    return set_err(h, STATEKV_ERR_INVALID_ARG, "unknown layer %d", layer);
+  const LayerState& L = h->layers[layer];
+  if (k) *k = L.kd;
+  if (v) *v = L.vd;
+  if (pos) *pos = L.posd;
+  if (len) *len = L.frames * h->T;
+  return STATEKV_OK;
+}
+
+int statekv_get_step_stats(statekv_t h, const float** lse, const float** pool_score, int* pool_len) {
+  if (!h) return set_err(nullptr, STATEKV_ERR_INVALID_ARG, "null handle");
+  if (lse) *lse = h->lse;
+  if (pool_score) *pool_score = h->pool_score;
+  if (pool_len) *pool_len = h->last_pool_len;
+  return STATEKV_OK;
+}
+
+int statekv_profile_enable(statekv_t h, int on) {
+  if (!h) return set_err(nullptr, STATEKV_ERR_INVALID_ARG, "null handle");
+  if (!on) {
+    for (auto& r : h->recs) {
+      h->ev_free.push_back(r.a);
+      h->ev_free.push_back(r.b);
+    }
+    h->recs.clear();
+  }
+  h->prof = on != 0;
+  return STATEKV_OK;
+}
+
+int statekv_profile_read(statekv_t h, double* ms, long long* launches) {
+  if (!h) return set_err(nullptr, STATEKV_ERR_INVALID_ARG, "null handle");
+  double acc[STATEKV_N_STAGES] = {0};
+  long long cnt[STATEKV_N_STAGES] = {0};
+  int rc = STATEKV_OK;
+  for (auto& r : h->recs) {
+    float t = 0.f;
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&t, r.a, r.b);
+    if (e != cudaSuccess && rc == STATEKV_OK)
+      rc = set_err(h, STATEKV_ERR_CUDA, "event timing failed: %s", cudaGetErrorString(e));
+    acc[r.stage] += t;
+    cnt[r.stage] += 1;
+    h->ev_free.push_back(r.a);
+    h->ev_free.push_back(r.b);
+  }
+  h->recs.clear();
+  for (int i = 0; i < STATEKV_N_STAGES; ++i) {
+    if (ms) ms[i] = acc[i];
+    if (launches) launches[i] = cnt[i];
+  }
+  return rc;
+}
+
+long long statekv_kernel_launches(statekv_t h) { return h ? h->launches : 0; }
+
+int statekv_frames(statekv_t h, int layer) {
+  if (!h || layer < 0 || (size_t)layer >= h->layers.size()) return 0;
+  return h->layers[layer].frames;
+}
+
+int statekv_destroy(statekv_t h) {
+  if (!h) return set_err(nullptr, STATEKV_ERR_INVALID_ARG, "null handle");
+  cudaDeviceSynchronize();
+  for (auto& r : h->recs) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  for (cudaEvent_t e : h->ev_free) cudaEventDestroy(e);
+  for (void* p : h->allocs) cudaFree(p);
+  delete h;
+  return STATEKV_OK;
+}
+
+const char* statekv_last_error(statekv_t h) {
+  return h ? h->err.c_str() : g_free_error.c_str();
+}
+
+int full_causal_prefill_batched(const void* q, const void* k, const void* v, int n_seq, int n_tokens,
+                                int Hq, int Hkv, int d, int dtype, void* out, float* lse, void* stream) {
+  if (!q || !k || !v || !out) return set_err(nullptr, STATEKV_ERR_INVALID_ARG, "null pointer");
+  if (n_seq < 1 || n_tokens < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv)
+    return set_err(nullptr, STATEKV_ERR_INVALID_ARG, "bad shape");
+  if (dtype != STATEKV_BF16 && dtype != STATEKV_F32)
+    return set_err(nullptr, STATEKV_ERR_INVALID_ARG, "bad dtype %d", dtype);
+  if (d != 64 && d != 128) return set_err(nullptr, STATEKV_ERR_UNSUPPORTED, "head dim %d", d);
+  if (n_tokens == 0) return STATEKV_OK;
+  skv::AttnArgs aa{};
+  aa.q = q;
+  aa.q_s = (long long)n_tokens * Hq * d;
+  aa.q_row = Hq * d;
+  aa.ka = k;
+  aa.va = v;
+  aa.a_s = 0;
+  aa.a_g = 0;
+  aa.m = 0;
+  aa.kb = k;
+  aa.vb = v;
+  aa.b_s = (long long)n_tokens * Hkv * d;
+  aa.b_row = Hkv * d;
+  aa.nb = n_tokens;
+  aa.out = out;
+  aa.lse = lse;
+  aa.lse_s = (long long)Hq * n_tokens;
+  aa.n_rows = n_tokens;
+  aa.Hq = Hq;
+  aa.Hkv = Hkv;
+  aa.causal = 1;
+  aa.scale_log2 = skv::kLog2e / sqrtf((float)d);
+  cudaError_t e = skv::launch_attn_simt(aa, dtype, d, n_seq, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess)
+    return set_err(nullptr, STATEKV_ERR_CUDA, "attention launch failed: %s", cudaGetErrorString(e));
+  return STATEKV_OK;
+}
+
+int full_causal_prefill(const void* q, const void* k, const void* v, int n_tokens, int Hq, int Hkv, int d,
+                        int dtype, void* out, float* lse, void* stream) {
+  return full_causal_prefill_batched(q, k, v, 1, n_tokens, Hq, Hkv, d, dtype, out, lse, stream);
+}
+
+}  // extern "C"

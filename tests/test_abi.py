@@ -1,0 +1,74 @@
+"""The C-ABI library loads on a machine without a GPU and exports every
+function that include/*.h declares; argument errors that the host catches
+before touching the device return the documented status codes."""
+
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+DECL = re.compile(r"^\s*(?:int|const\s+char\s*\*|int64_t|long long)\s+\**(\w+)\s*\(", re.M)
+
+
+def declared_functions():
+    names = []
+    for hdr in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(hdr).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += DECL.findall(text)
+    return names
+
+
+def test_header_declares_boundary():
+    names = set(declared_functions())
+    for required in ["statekv_create", "statekv_prefill_frame", "statekv_get_compressed",
+                     "statekv_get_detailed", "statekv_destroy", "statekv_last_error",
+                     "full_causal_prefill"]:
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    from kv_cache_selection_b200 import statekv as S
+    missing = [n for n in declared_functions() if not hasattr(S.lib, n)]
+    assert not missing, f"not exported: {missing}"
+
+
+def test_host_side_argument_errors():
+    from kv_cache_selection_b200 import statekv as S
+    h = ctypes.c_void_p()
+    # Hq not a multiple of Hkv
+    assert S.lib.statekv_create(ctypes.byref(h), 3, 2, 64, 16, 32, 8, 0, 0, 0) == -1
+    assert b"Hkv" in S.lib.statekv_last_error(None)
+    # unsupported head dim
+    assert S.lib.statekv_create(ctypes.byref(h), 2, 1, 96, 16, 32, 8, 0, 0, 0) == -2
+    # bad enums
+    assert S.lib.statekv_create(ctypes.byref(h), 2, 1, 64, 16, 32, 8, 7, 0, 0) == -1
+    assert S.lib.statekv_create(ctypes.byref(h), 2, 1, 64, 16, 32, 8, 0, 5, 0) == -1
+    assert S.lib.statekv_create(ctypes.byref(h), 2, 1, 64, 16, 32, 8, 0, 0, 9) == -1
+    # negative budget, empty frames
+    assert S.lib.statekv_create(ctypes.byref(h), 2, 1, 64, 16, -1, 8, 0, 0, 0) == -1
+    assert S.lib.statekv_create(ctypes.byref(h), 2, 1, 64, 0, 32, 8, 0, 0, 0) == -1
+    # null handle pointer and null handle
+    assert S.lib.statekv_create(None, 2, 1, 64, 16, 32, 8, 0, 0, 0) == -1
+    assert S.lib.statekv_prefill_frame(None, 0, None, None, None, None, None, None) == -1
+    assert S.lib.statekv_destroy(None) == -1
+    assert h.value is None
+    # full_causal_prefill argument checks
+    assert S.lib.full_causal_prefill(None, None, None, 4, 2, 1, 64, 0, None, None, None) == -1
+    assert S.lib.statekv_frames(None, 0) == 0
+
+
+def test_binding_refuses_missing_library(tmp_path, monkeypatch):
+    """No fallback: the binding raises if the library is absent."""
+    import importlib
+    import sys
+    monkeypatch.setenv("STATEKV_LIB", str(tmp_path / "nope.so"))
+    sys.modules.pop("kv_cache_selection_b200.statekv", None)
+    with pytest.raises(ImportError):
+        importlib.import_module("kv_cache_selection_b200.statekv")
+    monkeypatch.delenv("STATEKV_LIB")
+    sys.modules.pop("kv_cache_selection_b200.statekv", None)
+    importlib.import_module("kv_cache_selection_b200.statekv")

@@ -1,0 +1,241 @@
+"""GPU parity of the StateKV step (C ABI through the Python binding) against
+the float64 oracle, per step ("teacher forced"): at every checked frame the
+oracle starts from the GPU's own compressed state C_{n-1}, runs one step on the
+same inputs and is compared with the GPU's out, lse, pool scores and kept set.
+D and the rows of C are checked bit-exact against the source tokens.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import statekv_oracle as O
+from kv_cache_selection_b200 import synthetic as Syn
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+cuda = pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
+
+
+def _skv():
+    from kv_cache_selection_b200 import statekv
+    return statekv
+
+
+def _clone_C(C):
+    return {k: (v.clone() if isinstance(v, torch.Tensor) else v) for k, v in C.items()}
+
+
+def run_stream_parity(wl, n_frames, check, B=None, mask="frame_causal", select="global",
+                      n_streams=1, layer=0):
+    """Run n_frames on the GPU; teacher-forced oracle check at frames in `check`."""
+    S = _skv()
+    B = wl.B if B is None else B
+    dev = torch.device("cuda")
+    h = S.StateKV(wl.Hq, wl.Hkv, wl.d, wl.T, B, max_frames=n_frames, dtype=wl.dtype,
+                  mask=mask, select=select, n_streams=n_streams)
+    omask = O.MASK_FRAME_CAUSAL if mask == "frame_causal" else O.MASK_FRAME_BIDIR
+    osel = O.SELECT_GLOBAL if select == "global" else O.SELECT_PER_KV_HEAD
+    G = wl.Hq // wl.Hkv
+    mass = wl.Hq * wl.T if select == "global" else G * wl.T
+    all_frames = [[Syn.gen_frame(wl, n, layer=layer, stream=s) for s in range(n_streams)]
+                  for n in range(n_frames)]
+    report = dict(near_boundary=0, checked=0, max_rel_l2=0.0, max_score_rel=0.0)
+    for n in range(n_frames):
+        fr = all_frames[n]
+        stack = (lambda i: torch.stack([f[i] for f in fr]).to(dev)) if n_streams > 1 else \
+                (lambda i: fr[0][i].to(dev))
+        q, k, v, pos = stack(0), stack(1), stack(2), stack(3)
+        do_check = n in check
+        C_before = _clone_C(h.get_compressed(layer)) if (do_check and n > 0) else None
+        out = h.prefill_frame(layer, q, k, v, pos)
+        if not do_check:
+            continue
+        torch.cuda.synchronize()
+        stats = {k2: (v2.clone() if isinstance(v2, torch.Tensor) else v2) for k2, v2 in h.step_stats().items()}
+        C_after = _clone_C(h.get_compressed(layer))
+        for s in range(n_streams):
+            st = P.oracle_state_from_gpu(C_before, s) if C_before is not None else \
+                O.LayerState.empty(wl.Hkv, wl.d)
+            qs, ks, vs, ps = fr[s]
+            new, res = O.statekv_step(st, qs, ks, vs, ps.numpy(), B, omask, osel)
+            o_s = out[s] if n_streams > 1 else out
+            rel, _ = P.check_out(o_s, res["out"], wl.dtype, what=f"frame {n} stream {s} out")
+            report["max_rel_l2"] = max(report["max_rel_l2"], rel)
+            P.check_lse(stats["lse"][s], res["lse"], wl.dtype)
+            L = stats["pool_len"]
+            assert L == st.m + wl.T
+            rows = slice(0, 1) if select == "global" else slice(0, wl.Hkv)
+            sr = P.check_scores(stats["pool_score"][s, rows, :L], res["score"][rows], mass)
+            report["max_score_rel"] = max(report["max_score_rel"], sr)
+            assert C_after["len"] == min(B, st.m + wl.T)
+            for g in range(wl.Hkv):
+                got_pos = C_after["pos"][s, g, :C_after["len"]].cpu().numpy()
+                report["near_boundary"] += P.check_selection(
+                    got_pos, res["kept"][g], res["score"][g], res["pool_pos"][g], B)
+                # kept rows are bit-exact copies of the source tokens
+                pool_k = np.concatenate([st.K_C[g], O.to_f64(ks)[:, g]]) if st.m else O.to_f64(ks)[:, g]
+                pool_v = np.concatenate([st.V_C[g], O.to_f64(vs)[:, g]]) if st.m else O.to_f64(vs)[:, g]
+                where = {int(p): j for j, p in enumerate(res["pool_pos"][g])}
+                sel = [where[int(p)] for p in got_pos]
+                np.testing.assert_array_equal(O.to_f64(C_after["k"][s, g, :len(sel)]), pool_k[sel])
+                np.testing.assert_array_equal(O.to_f64(C_after["v"][s, g, :len(sel)]), pool_v[sel])
+                # stored scores are the pool scores of the kept candidates
+                got_sc = C_after["score"][s, g, :len(sel)].cpu().numpy()
+                np.testing.assert_array_equal(
+                    got_sc, stats["pool_score"][s, 0 if select == "global" else g, sel].cpu().numpy())
+            report["checked"] += 1
+    # D holds every frame token unmodified, in arrival order
+    torch.cuda.synchronize()
+    D = h.get_detailed(layer)
+    assert D["len"] == n_frames * wl.T
+    for s in range(n_streams):
+        Kc = torch.cat([all_frames[n][s][1] for n in range(n_frames)]).transpose(0, 1)
+        Vc = torch.cat([all_frames[n][s][2] for n in range(n_frames)]).transpose(0, 1)
+        pc = torch.cat([all_frames[n][s][3] for n in range(n_frames)])
+        assert torch.equal(D["k"][s, :, :D["len"]].cpu(), Kc)
+        assert torch.equal(D["v"][s, :, :D["len"]].cpu(), Vc)
+        assert torch.equal(D["pos"][s, :D["len"]].cpu(), pc)
+    h.close()
+    return report
+
+
+@cuda
+def test_tiny_f32_every_frame():
+    wl = Syn.workload("tiny")
+    r = run_stream_parity(wl, wl.frames, check=range(wl.frames))
+    assert r["checked"] == wl.frames
+
+
+@cuda
+def test_tiny_no_eviction_equals_full_causal():
+    """B=128 >= 8*16 tokens: the streamed outputs equal causal attention over
+    all 128 tokens (the oracle's quadratic comparator)."""
+    S = _skv()
+    wl = Syn.workload("tiny_noevict")
+    frames = Syn.gen_frames(wl)
+    h = S.StateKV(wl.Hq, wl.Hkv, wl.d, wl.T, wl.B, wl.frames, dtype="f32")
+    outs = [h.prefill_frame(0, *(t.cuda() for t in f)).cpu() for f in frames]
+    ref, _ = O.causal_attention(torch.cat([f[0] for f in frames]), torch.cat([f[1] for f in frames]),
+                                torch.cat([f[2] for f in frames]))
+    P.check_out(torch.cat(outs), ref, "f32")
+    C = h.get_compressed(0)
+    assert C["len"] == 128
+    assert torch.equal(C["pos"][0, 0].cpu(), torch.arange(128, dtype=torch.int32))
+
+
+@cuda
+@pytest.mark.parametrize("mask,select", [("frame_causal", "per_kv_head"), ("frame_bidir", "global"),
+                                         ("frame_bidir", "per_kv_head")])
+def test_modes_small(mask, select):
+    wl = Syn.workload("1b_layer", Hq=6, Hkv=2, d=64, T=24, B=40, frames=7, n_sinks=3)
+    r = run_stream_parity(wl, wl.frames, check=range(wl.frames), mask=mask, select=select)
+    assert r["checked"] == wl.frames
+
+
+@cuda
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d", [64, 128])
+def test_ragged_shapes(dtype, d):
+    """T and B not multiples of any tile; GQA group of 7."""
+    wl = Syn.workload("1b_layer", Hq=7, Hkv=1, d=d, T=37, B=90, frames=6, n_sinks=4, dtype=dtype)
+    run_stream_parity(wl, wl.frames, check=range(wl.frames))
+
+
+@cuda
+def test_zero_budget():
+    wl = Syn.workload("1b_layer", Hq=4, Hkv=2, d=64, T=16, B=0, frames=3, n_sinks=2)
+    r = run_stream_parity(wl, wl.frames, check=range(wl.frames), B=0)
+    assert r["checked"] == 3
+
+
+@cuda
+def test_1b_layer_all_frames():
+    wl = Syn.workload("1b_layer")
+    r = run_stream_parity(wl, wl.frames, check=range(wl.frames))
+    assert r["checked"] == wl.frames
+
+
+@cuda
+def test_8b_layer_full_size_sampled_frames():
+    """The 8B-class layer at full size (512 frames, B=4096): per-step parity on
+    sampled frames across the fill-up phase and the steady state."""
+    wl = Syn.workload("8b_layer")
+    r = run_stream_parity(wl, wl.frames, check={0, 1, 15, 16, 17, 100, 511})
+    assert r["checked"] == 7
+
+
+@cuda
+def test_batched_streams_match_single():
+    """Four streams in one handle give exactly what four single-stream handles
+    give (the streams share no state)."""
+    S = _skv()
+    wl = Syn.workload("1b_layer", Hq=14, Hkv=2, d=64, T=64, B=192, frames=6)
+    dev = torch.device("cuda")
+    hb = S.StateKV(wl.Hq, wl.Hkv, wl.d, wl.T, wl.B, wl.frames, dtype="bf16", n_streams=4)
+    singles = [S.StateKV(wl.Hq, wl.Hkv, wl.d, wl.T, wl.B, wl.frames, dtype="bf16") for _ in range(4)]
+    for n in range(wl.frames):
+        fr = [Syn.gen_frame(wl, n, stream=s) for s in range(4)]
+        ob = hb.prefill_frame(0, *(torch.stack([f[i] for f in fr]).to(dev) for i in range(4)))
+        for s in range(4):
+            os_ = singles[s].prefill_frame(0, *(t.to(dev) for t in fr[s]))
+            assert torch.equal(ob[s], os_)
+    Cb = hb.get_compressed(0)
+    for s in range(4):
+        Cs = singles[s].get_compressed(0)
+        assert torch.equal(Cb["pos"][s], Cs["pos"][0])
+        assert torch.equal(Cb["k"][s], Cs["k"][0])
+
+
+@cuda
+def test_batched_streams_parity():
+    wl = Syn.workload("1b_layer", Hq=14, Hkv=2, d=64, T=64, B=192, frames=5)
+    run_stream_parity(wl, wl.frames, check=range(wl.frames), n_streams=3)
+
+
+@cuda
+def test_capacity_and_argument_errors():
+    S = _skv()
+    h = S.StateKV(2, 1, 64, 16, 32, max_frames=2, dtype="f32")
+    wl = Syn.workload("tiny")
+    for n in range(2):
+        h.prefill_frame(0, *(t.cuda() for t in Syn.gen_frame(wl, n)))
+    with pytest.raises(S.StateKVError) as e:
+        h.prefill_frame(0, *(t.cuda() for t in Syn.gen_frame(wl, 2)))
+    assert e.value.code == -3
+    assert h.frames(0) == 2
+    # a different layer is independent
+    h.prefill_frame(3, *(t.cuda() for t in Syn.gen_frame(wl, 0)))
+    assert h.frames(3) == 1 and h.frames(1) == 0
+    with pytest.raises(S.StateKVError):
+        h.get_compressed(1)  # never called (allocated by the resize, not ready)
+    with pytest.raises(ValueError):
+        h.prefill_frame(0, *(t.cuda() for t in Syn.gen_frame(Syn.workload("1b_layer"), 0)))
+
+
+@cuda
+@pytest.mark.parametrize("dtype,N,Hq,Hkv,d", [("f32", 100, 2, 1, 64), ("bf16", 333, 14, 2, 64),
+                                             ("bf16", 300, 28, 4, 128), ("f32", 257, 4, 4, 128)])
+def test_full_causal_prefill_small(dtype, N, Hq, Hkv, d):
+    S = _skv()
+    wl = Syn.workload("1b_layer", Hq=Hq, Hkv=Hkv, d=d, T=64, dtype=dtype)
+    q, k, v = Syn.gen_tokens(wl, N)
+    out, lse = S.full_causal_prefill(q.cuda(), k.cuda(), v.cuda())
+    ref_out, ref_lse = O.causal_attention(q, k, v)
+    P.check_out(out, ref_out, dtype)
+    P.check_lse(lse, ref_lse, dtype)
+
+
+@cuda
+def test_full_causal_prefill_large_sampled_rows():
+    """8B layer shape over 16 frames x 256 tokens; rows sampled across tiles."""
+    S = _skv()
+    wl = Syn.workload("8b_layer")
+    N = 16 * 256
+    q, k, v = Syn.gen_tokens(wl, N)
+    out, lse = S.full_causal_prefill(q.cuda(), k.cuda(), v.cuda())
+    rows = [0, 1, 127, 128, 129, 2047, 2048, 3000, N - 2, N - 1]
+    ref_out, ref_lse = O.causal_attention_rows(q, k, v, rows)
+    P.check_out(out[rows], ref_out, "bf16")
+    P.check_lse(lse[:, rows], ref_lse, "bf16")
