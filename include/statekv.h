@@ -196,6 +196,41 @@ int full_causal_prefill_batched(const void* q, const void* k, const void* v, int
                                 int n_tokens, int Hq, int Hkv, int d, int dtype, void* out,
                                 float* lse, void* stream);
 
+/* One StateKV step (same computation as statekv_prefill_frame for S = 1) that
+ * allocates no device memory.  The paper has no counterpart: this is a
+ * deployment variant for callers that cannot call cudaMalloc when they run the
+ * step, e.g. a server that has already reserved nearly all GPU memory for its
+ * own pool, or a latency-critical loop that cannot afford cudaMalloc's
+ * implicit device-wide synchronisation.
+ *
+ * The caller owns every tensor (device pointers, 16-byte aligned):
+ *   q [T][Hq][d], k,v [T][Hkv][d], pos [T]        the frame (as prefill_frame);
+ *   kc,vc [Hkv][B][d], posc [Hkv][B], m            C_{n-1}: its first m rows;
+ *   out [T][Hq][d]                                 attention output;
+ *   kc_new,vc_new [Hkv][B][d], posc_new, scorec_new [Hkv][B]
+ *                                                  C_n (min(B, m+T) rows); must
+ *                                                  not alias kc/vc;
+ *   kd,vd [Hkv][max_tok][d], posd [max_tok]        D; the frame is appended at
+ *                                                  token d_len (d_len+T <= max_tok).
+ * Per-step scratch lives in one file-scope device array of 1 MiB per device
+ * (lse [Hq][T], partial and pool scores [Hkv][B+T], kept list [Hkv][B], each
+ * rounded up to 256 bytes); shapes that need more are rejected with
+ * STATEKV_ERR_UNSUPPORTED and a message naming the size.  Nothing in the
+ * scratch must start at zero (each call writes what it reads).  The array is
+ * shared by every call on the device and keeps the last call's contents, so
+ * calls whose work overlaps on the GPU (different streams, or threads using
+ * this entry point concurrently) race; order them on one stream.  The first
+ * call on each device looks up the array's device address (with that device
+ * current); make that first call before any stream capture.
+ * Errors (message in statekv_last_error(NULL)): INVALID_ARG, UNSUPPORTED,
+ * CAPACITY, CUDA. */
+int statekv_step_noalloc(int Hq, int Hkv, int d, int T, int B, int dtype, int mask_mode,
+                         int select_mode, const void* q, const void* k, const void* v,
+                         const int32_t* pos, const void* kc, const void* vc,
+                         const int32_t* posc, int m, void* out, void* kc_new, void* vc_new,
+                         int32_t* posc_new, float* scorec_new, void* kd, void* vd,
+                         int32_t* posd, int d_len, int max_tok, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

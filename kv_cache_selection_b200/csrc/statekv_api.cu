@@ -199,6 +199,10 @@ int launch_err(statekv_t h, cudaError_t e, const char* what) {
 
 }  // namespace
 
+namespace skv {
+void set_free_error(const char* msg) { g_free_error = msg; }
+}  // namespace skv
+
 extern "C" {
 
 int statekv_create_batched(statekv_t* out, int n_streams, int Hq, int Hkv, int d, int T, int B,

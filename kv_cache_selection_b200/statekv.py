@@ -51,6 +51,7 @@ _SIGS = {
     "statekv_kernel_launches": (ctypes.c_longlong, [_vp]),
     "statekv_destroy": (_i, [_vp]),
     "statekv_last_error": (ctypes.c_char_p, [_vp]),
+    "statekv_step_noalloc": (_i, [_i] * 8 + [_vp] * 7 + [_i] + [_vp] * 8 + [_i, _i, _vp]),
     "full_causal_prefill": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp]),
     "full_causal_prefill_batched": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp]),
 }
