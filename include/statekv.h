@@ -169,6 +169,12 @@ int statekv_profile_read(statekv_t h, double* ms, long long* launches);
 /* Number of kernels this handle has launched since it was created. */
 long long statekv_kernel_launches(statekv_t h);
 
+/* Device-side status of the handle's kernels: *code = 0, or the first error a
+ * kernel recorded since the last call (a pipeline wait that exceeded its time
+ * limit; the kernel then abandoned its tile and exited cleanly, so results of
+ * that step are invalid).  Synchronises the device, then resets the word. */
+int statekv_device_status(statekv_t h, int* code);
+
 /* Frames processed so far on a layer (0 for a layer never called). */
 int statekv_frames(statekv_t h, int layer);
 

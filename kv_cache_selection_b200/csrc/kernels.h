@@ -1,6 +1,7 @@
 // Internal launchers of libstatekv (not part of the C ABI).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -14,6 +15,27 @@ cudaError_t launch_attn_simt(const AttnArgs& a, int dtype, int d, int S, cudaStr
 cudaError_t launch_score_simt(const ScoreArgs& a, int dtype, int d, int S, cudaStream_t st);
 cudaError_t launch_select(const SelectArgs& a, int S, cudaStream_t st);
 cudaError_t launch_gather(const GatherArgs& a, int n_sm, cudaStream_t st);
+
+// bf16 4-D tiled TMA map, 128-byte swizzle, zero fill out of bounds.  dims[0]
+// is the innermost (contiguous) extent in elements; strides_bytes[i] is the
+// byte stride of dims[i+1].  Returns 0 or a CUresult.
+int encode_tmap_bf16_4d(CUtensorMap* map, const void* base, const uint64_t dims[4],
+                        const uint64_t strides_bytes[3], const uint32_t box[4]);
+
+// Tensor-core score pass (bf16): the three maps cover q [S][T][Hq][d],
+// K_C [S][Hkv][B][d] and the frame keys [S][T][Hkv][d], boxes of 64 x 128 rows.
+struct ScoreTcArgs {
+  const float* lse;  // [S][Hq][T] natural log
+  long long lse_s;
+  float* part;       // [S][Hkv][pool]
+  long long part_s;
+  int part_g;
+  int m, T, Hq, Hkv, causal, n_c_tiles, n_f_tiles, S;
+  float scale_log2;
+  int* err;          // device error word (timeouts)
+};
+cudaError_t launch_score_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kc, const CUtensorMap& tm_kf,
+                            const ScoreTcArgs& a, int d, cudaStream_t st);
 
 // Message for statekv_last_error(NULL) (errors of calls without a handle).
 void set_free_error(const char* msg);

@@ -1,0 +1,268 @@
+// Score pass on the 5th-generation tensor cores (bf16 in, f32 accumulate).
+//
+// The score of pool candidate j is the sum, over the frame's query rows i and
+// the query heads h of its KV group, of the normalised attention weight
+// P_hij = exp(s_hij - lse_hi) ("Linear Scaling Video VLMs for Long Video
+// Understanding", P1 section 方法步骤详情: sum the attention weights over all
+// queries; P2 A.3 "Kernel considerations": fused attention kernels do not
+// expose the weights, so they are recomputed here from the row statistics and
+// never written to memory).
+//
+// Transposed formulation: one CTA owns 128 candidates (keys) of one KV group
+// and computes S^T = K Q^T, 128 keys (TMEM lanes) x 128 query rows (TMEM
+// columns) per chunk, streaming the group's G*T query rows through a TMA ring.
+// Each epilogue thread owns one key's TMEM lane, so the column sum of P is a
+// private running sum: no shuffles, no atomics, deterministic.
+//
+// Warp roles (320 threads): warp 0 TMA producer, warp 1 TMEM allocator + MMA
+// issuer, warps 2..9 epilogue (two warpgroups split each chunk's columns).
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_common.cuh"
+
+namespace skv {
+namespace {
+using namespace tc;
+
+constexpr int kStages = 4;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+
+template <int D>
+struct Smem {
+  static constexpr int kAtoms = D / 64;                  // 64-element (128-byte) swizzle atoms
+  static constexpr int kAtomBytes = 128 * 128;           // 128 rows x 128 bytes
+  static constexpr int kTileBytes = kAtoms * kAtomBytes;
+  static constexpr int kK = 0;
+  static constexpr int kQ = kK + kTileBytes;
+  static constexpr int kLse = kQ + kStages * kTileBytes;  // per epilogue warp: 64 floats
+  static constexpr int kRed = kLse + kEpiWarps * 64 * 4;  // 128 floats
+  static constexpr int kBar = kRed + 128 * 4;
+  // k_full, q_full[kStages], q_empty[kStages], acc_full[2], acc_empty[2], done
+  static constexpr int kNumBars = 1 + 2 * kStages + 4 + 1;
+  static constexpr int kTmemSlot = kBar + kNumBars * 8;
+  static constexpr int kAbort = kTmemSlot + 4;
+  static constexpr int kBytes = kAbort + 4;
+  static constexpr int kAlloc = kBytes + 1024;            // room to align the base to 1024
+};
+
+// Bounded wait used on the teardown path only: ignores the abort flag.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, int* err) {
+  const unsigned long long t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      atomicCAS(err, 0, kErrWaitDrain);
+      return;
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kc,
+                    const __grid_constant__ CUtensorMap tm_kf, ScoreTcArgs a) {
+  using L = Smem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int s = blockIdx.z, g = blockIdx.y, tile = blockIdx.x;
+  const bool is_c = tile < a.n_c_tiles;
+  const int r0 = is_c ? tile * 128 : (tile - a.n_c_tiles) * 128;  // first C row / frame token
+  const int G = a.Hq / a.Hkv;
+  const int n_ic = (a.T + 127) / 128;
+  // frame-causal: frame token t is seen only by query rows i >= t, so chunks
+  // ending before r0 hold nothing visible for this tile
+  const int ic_min = (!is_c && a.causal) ? r0 / 128 : 0;
+  const int per_head = n_ic - ic_min;
+  const int n_chunks = G * per_head;
+
+  const uint32_t bar_k = sb + L::kBar;
+  auto bar_qfull = [&](int st) { return sb + L::kBar + 8u * (1 + st); };
+  auto bar_qempty = [&](int st) { return sb + L::kBar + 8u * (1 + kStages + st); };
+  auto bar_accfull = [&](int b) { return sb + L::kBar + 8u * (1 + 2 * kStages + b); };
+  auto bar_accempty = [&](int b) { return sb + L::kBar + 8u * (3 + 2 * kStages + b); };
+  const uint32_t bar_done = sb + L::kBar + 8u * (5 + 2 * kStages);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_k, 1);
+    for (int st = 0; st < kStages; ++st) {
+      mbar_init(bar_qfull(st), 1);
+      mbar_init(bar_qempty(st), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_accfull(b), 1);
+      mbar_init(bar_accempty(b), kEpiWarps);
+    }
+    mbar_init(bar_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 256);  // two 128-column f32 accumulators
+    tmem_relinquish();
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(is_c ? &tm_kc : &tm_kf);
+      mbar_arrive_expect_tx(bar_k, L::kTileBytes);
+      for (int at = 0; at < L::kAtoms; ++at) {
+        if (is_c) tma_load_4d(sb + L::kK + at * L::kAtomBytes, &tm_kc, bar_k, at * 64, r0, g, s);
+        else tma_load_4d(sb + L::kK + at * L::kAtomBytes, &tm_kf, bar_k, at * 64, g, r0, s);
+      }
+      int issued = 0;
+      for (int c = 0; c < n_chunks; ++c) {
+        const int st = c % kStages;
+        if (!mbar_wait(bar_qempty(st), ((c / kStages) & 1) ^ 1, a.err, kErrWaitEmpty, abort_flag)) break;
+        const int h = g * G + c / per_head;
+        const int i0 = (ic_min + c % per_head) * 128;
+        mbar_arrive_expect_tx(bar_qfull(st), L::kTileBytes);
+        for (int at = 0; at < L::kAtoms; ++at)
+          tma_load_4d(sb + L::kQ + st * L::kTileBytes + at * L::kAtomBytes, &tm_q, bar_qfull(st), at * 64, h,
+                      i0, s);
+        issued = c + 1;
+      }
+      // every armed load must land before the CTA may exit
+      drain_wait(bar_k, 0, a.err);
+      for (int c = (issued > kStages ? issued - kStages : 0); c < issued; ++c)
+        drain_wait(bar_qfull(c % kStages), (c / kStages) & 1, a.err);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(128, 128, false, false);
+      bool ok = mbar_wait(bar_k, 0, a.err, kErrWaitLoad, abort_flag);
+      for (int c = 0; ok && c < n_chunks; ++c) {
+        const int st = c % kStages, buf = c & 1;
+        if (!mbar_wait(bar_qfull(st), (c / kStages) & 1, a.err, kErrWaitLoad, abort_flag)) break;
+        if (!mbar_wait(bar_accempty(buf), ((c >> 1) & 1) ^ 1, a.err, kErrWaitAccFree, abort_flag)) break;
+        fence_after_sync();
+        const uint32_t qbase = sb + L::kQ + st * L::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::kAtomBytes + (kk & 3) * 32;
+          mma_ss(tmem + buf * 128, sdesc_sw128(sb + L::kK + off, 16, 1024), sdesc_sw128(qbase + off, 16, 1024),
+                 idesc, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar_qempty(st));
+        mma_commit(bar_accfull(buf));
+      }
+      mma_commit(bar_done);
+      drain_wait(bar_done, 0, a.err);
+    }
+    __syncwarp();
+  } else {
+    const int ew = warp - 2;              // 0..7
+    const int quarter = warp & 3;         // TMEM lane quarter this warp may access
+    const int half = ew >> 2;             // which 64 columns of each chunk
+    const int row = quarter * 32 + lane;  // key row within the tile
+    const int key = r0 + row;
+    float* lse2 = reinterpret_cast<float*>(smem + L::kLse) + ew * 64;
+    float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+    bool ok = true;
+    for (int c = 0; c < n_chunks; ++c) {
+      const int buf = c & 1;
+      const int h = g * G + c / per_head;
+      const int i0 = (ic_min + c % per_head) * 128;
+      const int cbase = i0 + half * 64;
+      // this warp's 64 row statistics, in log2 units (+inf past the frame)
+      __syncwarp();
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int i = cbase + lane + 32 * u;
+        lse2[lane + 32 * u] = i < a.T ? a.lse[s * a.lse_s + (long long)h * a.T + i] * kLog2e : INFINITY;
+      }
+      __syncwarp();
+      uint32_t got = 1;
+      if (lane == 0) got = mbar_wait(bar_accfull(buf), (c >> 1) & 1, a.err, kErrWaitAcc, abort_flag) ? 1u : 0u;
+      got = __shfl_sync(0xffffffffu, got, 0);
+      if (!got) {
+        ok = false;
+        break;
+      }
+      fence_after_sync();
+      // some of this warp's columns precede some key of the tile (warp-uniform)
+      const bool diag = !is_c && a.causal && (cbase < r0 + 127);
+#pragma unroll
+      for (int q32 = 0; q32 < 2; ++q32) {
+        uint32_t r[32];
+        tmem_ld32(tmem_addr(tmem, quarter * 32, buf * 128 + half * 64 + q32 * 32), r);
+        tmem_ld_wait();
+        const float4* l4 = reinterpret_cast<const float4*>(lse2 + q32 * 32);
+#pragma unroll
+        for (int j4 = 0; j4 < 8; ++j4) {
+          const float4 lv = l4[j4];
+          float p0 = ex2_approx(fmaf(__uint_as_float(r[4 * j4 + 0]), a.scale_log2, -lv.x));
+          float p1 = ex2_approx(fmaf(__uint_as_float(r[4 * j4 + 1]), a.scale_log2, -lv.y));
+          float p2 = ex2_approx(fmaf(__uint_as_float(r[4 * j4 + 2]), a.scale_log2, -lv.z));
+          float p3 = ex2_approx(fmaf(__uint_as_float(r[4 * j4 + 3]), a.scale_log2, -lv.w));
+          if (diag) {
+            const int i = cbase + q32 * 32 + 4 * j4;  // frame token `key` is seen by rows i >= key
+            p0 = key <= i + 0 ? p0 : 0.f;
+            p1 = key <= i + 1 ? p1 : 0.f;
+            p2 = key <= i + 2 ? p2 : 0.f;
+            p3 = key <= i + 3 ? p3 : 0.f;
+          }
+          acc0 += p0;
+          acc1 += p1;
+          acc2 += p2;
+          acc3 += p3;
+        }
+      }
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_accempty(buf));
+    }
+    // combine the two column halves of each key row
+    float tot = (acc0 + acc1) + (acc2 + acc3);
+    float* red = reinterpret_cast<float*>(smem + L::kRed);
+    if (half == 1) red[row] = tot;
+    named_bar_sync(1, 32 * kEpiWarps);
+    if (half == 0 && ok && !*abort_flag) {
+      tot += red[row];
+      const bool valid = is_c ? key < a.m : key < a.T;
+      if (valid) {
+        const int j = is_c ? key : a.m + key;
+        a.part[s * a.part_s + (long long)g * a.part_g + j] = tot;
+      }
+    }
+  }
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    fence_after_sync();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_score_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kc, const CUtensorMap& tm_kf,
+                            const ScoreTcArgs& a, int d, cudaStream_t st) {
+  const int n_tiles = a.n_c_tiles + a.n_f_tiles;
+  if (n_tiles == 0) return cudaSuccess;
+  dim3 grid(n_tiles, a.Hkv, a.S);
+  cudaError_t e;
+  if (d == 128) {
+    const int smem = Smem<128>::kAlloc;
+    if ((e = cudaFuncSetAttribute(score_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)))
+      return e;
+    score_tc_kernel<128><<<grid, kThreads, smem, st>>>(tm_q, tm_kc, tm_kf, a);
+  } else {
+    const int smem = Smem<64>::kAlloc;
+    if ((e = cudaFuncSetAttribute(score_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)))
+      return e;
+    score_tc_kernel<64><<<grid, kThreads, smem, st>>>(tm_q, tm_kc, tm_kf, a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace skv

@@ -53,6 +53,7 @@ struct statekv_handle {
   float* part = nullptr;        // [S][Hkv][B+T]
   float* pool_score = nullptr;  // [S][Hkv][B+T]
   int32_t* idx = nullptr;       // [S][Hkv][max(B,1)]
+  int* dev_err = nullptr;       // kernel error word (bounded-wait timeouts)
   // staging for statekv_prefill_frame_host (allocated on first use)
   void* stage_q = nullptr;
   void* stage_k = nullptr;
@@ -193,6 +194,27 @@ struct StageScope {
   }
 };
 
+// TMA maps of one step: q [S][T][Hq][d], K_C [S][Hkv][B][d], frame k [S][T][Hkv][d]
+int encode_step_maps(statekv_t h, const void* q, const void* kc, const void* k, CUtensorMap* tq,
+                     CUtensorMap* tkc, CUtensorMap* tkf) {
+  const uint64_t d = h->d, Hq = h->Hq, Hkv = h->Hkv, T = h->T, S = h->S;
+  const uint64_t B = std::max(h->B, 1);
+  const uint64_t dq[4] = {d, Hq, T, S};
+  const uint64_t sq[3] = {d * 2, Hq * d * 2, T * Hq * d * 2};
+  const uint32_t bq[4] = {64, 1, 128, 1};
+  const uint64_t dc[4] = {d, B, Hkv, S};
+  const uint64_t sc[3] = {d * 2, B * d * 2, Hkv * B * d * 2};
+  const uint32_t bc[4] = {64, 128, 1, 1};
+  const uint64_t dk[4] = {d, Hkv, T, S};
+  const uint64_t sk[3] = {d * 2, Hkv * d * 2, T * Hkv * d * 2};
+  int r;
+  if ((r = skv::encode_tmap_bf16_4d(tq, q, dq, sq, bq)) != 0 ||
+      (r = skv::encode_tmap_bf16_4d(tkc, kc, dc, sc, bc)) != 0 ||
+      (r = skv::encode_tmap_bf16_4d(tkf, k, dk, sk, bq)) != 0)
+    return set_err(h, STATEKV_ERR_CUDA, "TMA tensor map encoding failed (CUresult %d)", r);
+  return STATEKV_OK;
+}
+
 int launch_err(statekv_t h, cudaError_t e, const char* what) {
   return set_err(h, STATEKV_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString(e));
 }
@@ -234,7 +256,8 @@ int statekv_create_batched(statekv_t* out, int n_streams, int Hq, int Hkv, int d
   if ((rc = dev_alloc(h, (void**)&h->lse, (size_t)n_streams * Hq * T * 4)) ||
       (rc = dev_alloc(h, (void**)&h->part, (size_t)n_streams * Hkv * pool * 4)) ||
       (rc = dev_alloc(h, (void**)&h->pool_score, (size_t)n_streams * Hkv * pool * 4)) ||
-      (rc = dev_alloc(h, (void**)&h->idx, (size_t)n_streams * Hkv * std::max(B, 1) * 4))) {
+      (rc = dev_alloc(h, (void**)&h->idx, (size_t)n_streams * Hkv * std::max(B, 1) * 4)) ||
+      (rc = dev_alloc(h, (void**)&h->dev_err, 16))) {
     g_free_error = h->err;
     statekv_destroy(h);
     return rc;
@@ -333,7 +356,29 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
   sa.Hkv = Hkv;
   sa.causal = aa.causal;
   sa.scale_log2 = scale_log2;
-  {
+  if (h->dtype == STATEKV_BF16) {
+    CUtensorMap tq, tkc, tkf;
+    if ((rc = encode_step_maps(h, q, L->kc[cur], k, &tq, &tkc, &tkf))) return rc;
+    skv::ScoreTcArgs ta{};
+    ta.lse = h->lse;
+    ta.lse_s = aa.lse_s;
+    ta.part = h->part;
+    ta.part_s = sa.part_s;
+    ta.part_g = pool;
+    ta.m = m;
+    ta.T = T;
+    ta.Hq = Hq;
+    ta.Hkv = Hkv;
+    ta.causal = aa.causal;
+    ta.n_c_tiles = (m + 127) / 128;
+    ta.n_f_tiles = (T + 127) / 128;
+    ta.S = S;
+    ta.scale_log2 = scale_log2;
+    ta.err = h->dev_err;
+    StageScope sc(h, st, STATEKV_STAGE_SCORE);
+    if ((e = skv::launch_score_tc(tq, tkc, tkf, ta, d, st)) != cudaSuccess) return launch_err(h, e, "score");
+    sc.done();
+  } else {
     StageScope sc(h, st, STATEKV_STAGE_SCORE);
     if ((e = skv::launch_score_simt(sa, h->dtype, d, S, st)) != cudaSuccess) return launch_err(h, e, "score");
     sc.done();
@@ -500,6 +545,17 @@ int statekv_profile_read(statekv_t h, double* ms, long long* launches) {
 }
 
 long long statekv_kernel_launches(statekv_t h) { return h ? h->launches : 0; }
+
+int statekv_device_status(statekv_t h, int* code) {
+  if (!h || !code) return set_err(h, STATEKV_ERR_INVALID_ARG, "null argument");
+  int v = 0;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(&v, h->dev_err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(h->dev_err, 0, sizeof(int));
+  if (e != cudaSuccess) return set_err(h, STATEKV_ERR_CUDA, "status read failed: %s", cudaGetErrorString(e));
+  *code = v;
+  return STATEKV_OK;
+}
 
 int statekv_frames(statekv_t h, int layer) {
   if (!h || layer < 0 || (size_t)layer >= h->layers.size()) return 0;

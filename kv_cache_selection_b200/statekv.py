@@ -49,6 +49,7 @@ _SIGS = {
     "statekv_profile_enable": (_i, [_vp, _i]),
     "statekv_profile_read": (_i, [_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)]),
     "statekv_kernel_launches": (ctypes.c_longlong, [_vp]),
+    "statekv_device_status": (_i, [_vp, _ip]),
     "statekv_destroy": (_i, [_vp]),
     "statekv_last_error": (ctypes.c_char_p, [_vp]),
     "statekv_step_noalloc": (_i, [_i] * 8 + [_vp] * 7 + [_i] + [_vp] * 8 + [_i, _i, _vp]),
@@ -173,6 +174,12 @@ class StateKV:
         cnt = (ctypes.c_longlong * N_STAGES)()
         _check(lib.statekv_profile_read(self._h, ms, cnt), self._h)
         return {name: (ms[i], cnt[i]) for i, name in enumerate(STAGES) if name}
+
+    def device_status(self) -> int:
+        """0, or the first error code a kernel recorded (synchronises)."""
+        code = ctypes.c_int()
+        _check(lib.statekv_device_status(self._h, ctypes.byref(code)), self._h)
+        return code.value
 
     def kernel_launches(self) -> int:
         return lib.statekv_kernel_launches(self._h)

@@ -97,6 +97,7 @@ def run_stream_parity(wl, n_frames, check, B=None, mask="frame_causal", select="
         assert torch.equal(D["k"][s, :, :D["len"]].cpu(), Kc)
         assert torch.equal(D["v"][s, :, :D["len"]].cpu(), Vc)
         assert torch.equal(D["pos"][s, :D["len"]].cpu(), pc)
+    assert h.device_status() == 0
     h.close()
     return report
 
