@@ -1,0 +1,466 @@
+// Attention of the frame's queries over [C_{n-1}; frame] on the 5th-generation
+// tensor cores (bf16 in, f32 accumulate), with per-row log-sum-exp out.
+//
+// "Linear Scaling Video VLMs for Long Video Understanding", P1 section
+// 方法步骤详情: the current frame's queries attend over the concatenation of
+// the compressed memory and the current frame's tokens (softmax of the dot
+// products, times the values); the frame is causal inside (P1 section
+// 自注意力复杂度) and every compressed entry is visible.  The same kernel, with
+// an empty compressed state and the whole sequence as "frame", is the full
+// causal comparator.
+//
+// One CTA takes two 128-row query tiles (A, B) of one KV group and a range of
+// 128-key tiles.  Per key tile and query tile:
+//   S = Q K^T            tcgen05.mma, A = Q (smem), B = K (smem), D = S (TMEM)
+//   P = exp2(S*c - m)    softmax warpgroup: TMEM -> registers -> bf16 P back
+//                        into the same TMEM columns
+//   O += P V             tcgen05.mma with A = P read from TMEM, B = V (smem,
+//                        MN-major), D = O (TMEM)
+// The two softmax warpgroups alternate with the tensor core (while one
+// computes P, the other tile's MMAs run).  The running max is applied lazily:
+// O and the row sum are rescaled only when a row's max grows by more than 2^8,
+// so P stays below 256 and the result is exact up to rounding.  Key tiles are
+// split across CTAs to fill the SMs; each split writes (O/l, log2-sum-exp)
+// partials that attn_combine merges, or out and lse directly when unsplit.
+//
+// Warp roles (384 threads): warp 0 TMA producer, warp 1 TMEM allocator + MMA
+// issuer, warps 4..7 softmax of tile A, warps 8..11 softmax of tile B.
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_common.cuh"
+
+namespace skv {
+namespace {
+using namespace tc;
+
+constexpr int kSlots = 4;        // K/V ring slots (each one 128-key tile)
+constexpr int kThreads = 384;
+constexpr float kRescaleLog2 = 8.0f;
+
+template <int D>
+struct AttnSmem {
+  static constexpr int kAtoms = D / 64;
+  static constexpr int kAtomBytes = 128 * 128;
+  static constexpr int kTileBytes = kAtoms * kAtomBytes;  // 128 rows x D bf16
+  static constexpr int kQ = 0;                             // Q tiles A, B
+  static constexpr int kKV = 2 * kTileBytes;               // ring
+  static constexpr int kBar = kKV + kSlots * kTileBytes;
+  // q_full, kv_full[kSlots], kv_empty[kSlots], s_full[2], p_full[2], o_done[2], done
+  static constexpr int kNumBars = 1 + 2 * kSlots + 6 + 1;
+  static constexpr int kTmemSlot = kBar + kNumBars * 8;
+  static constexpr int kAbort = kTmemSlot + 4;
+  static constexpr int kBytes = kAbort + 4;
+  // at least 116 KB so that a second CTA (which would also need all 512 TMEM
+  // columns) never shares the SM
+  static constexpr int kAlloc = kBytes + 1024 > 116 * 1024 ? kBytes + 1024 : 116 * 1024;
+};
+
+struct TileInfo {
+  bool valid;
+  int h, i0, nk;  // head, first query row, key tiles it needs in total
+};
+
+__device__ __forceinline__ TileInfo tile_info(const AttnTcArgs& a, int g, int t) {
+  TileInfo ti;
+  const int G = a.Hq / a.Hkv;
+  ti.valid = t < G * a.n_it;
+  if (!ti.valid) t = 0;
+  ti.h = g * G + t / a.n_it;
+  ti.i0 = (t % a.n_it) * 128;
+  int nf = a.nF;
+  if (a.causal) {
+    const int i_max = min(ti.i0 + 127, a.T - 1);  // last row of the tile
+    nf = i_max / 128 + 1;                          // frame tiles holding tokens <= i_max
+  }
+  ti.nk = a.nC + nf;
+  return ti;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kc,
+                   const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_kf,
+                   const __grid_constant__ CUtensorMap tm_vf, AttnTcArgs a) {
+  using L = AttnSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // unit -> (stream, KV group, query-tile pair, key split)
+  int u = blockIdx.x;
+  const int sp = u % a.n_split;
+  u /= a.n_split;
+  const int pair = a.n_pairs - 1 - u % a.n_pairs;  // later query tiles (more keys) first
+  u /= a.n_pairs;
+  const int g = u % a.Hkv;
+  const int s = u / a.Hkv;
+  const TileInfo tA = tile_info(a, g, 2 * pair), tB = tile_info(a, g, 2 * pair + 1);
+  const int nk = max(tA.nk, tB.valid ? tB.nk : 0);
+  const int kb = sp * nk / a.n_split, ke = (sp + 1) * nk / a.n_split;
+  const int nA = max(0, min(ke, tA.nk) - kb);
+  const int nB = tB.valid ? max(0, min(ke, tB.nk) - kb) : 0;
+  const int n_load = max(nA, nB);
+
+  const uint32_t bar_q = sb + L::kBar;
+  auto bar_kvfull = [&](int sl) { return sb + L::kBar + 8u * (1 + sl); };
+  auto bar_kvempty = [&](int sl) { return sb + L::kBar + 8u * (1 + kSlots + sl); };
+  auto bar_sfull = [&](int x) { return sb + L::kBar + 8u * (1 + 2 * kSlots + x); };
+  auto bar_pfull = [&](int x) { return sb + L::kBar + 8u * (3 + 2 * kSlots + x); };
+  auto bar_odone = [&](int x) { return sb + L::kBar + 8u * (5 + 2 * kSlots + x); };
+  const uint32_t bar_done = sb + L::kBar + 8u * (7 + 2 * kSlots);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int sl = 0; sl < kSlots; ++sl) {
+      mbar_init(bar_kvfull(sl), 1);
+      mbar_init(bar_kvempty(sl), 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bar_sfull(x), 1);
+      mbar_init(bar_pfull(x), 4);
+      mbar_init(bar_odone(x), 1);
+    }
+    mbar_init(bar_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  // TMEM columns: S/P of tile A at 0, of tile B at 128, O of A at 256, O of B at 384
+  auto col_s = [](int x) { return (uint32_t)(x * 128); };
+  auto col_o = [](int x) { return (uint32_t)(256 + x * 128); };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      const int nq = (nA > 0 ? 1 : 0) + (nB > 0 ? 1 : 0);
+      if (nq) {
+        mbar_arrive_expect_tx(bar_q, nq * L::kTileBytes);
+        for (int at = 0; at < L::kAtoms; ++at) {
+          if (nA > 0) tma_load_4d(sb + L::kQ + at * L::kAtomBytes, &tm_q, bar_q, at * 64, tA.h, tA.i0, s);
+          if (nB > 0)
+            tma_load_4d(sb + L::kQ + L::kTileBytes + at * L::kAtomBytes, &tm_q, bar_q, at * 64, tB.h, tB.i0, s);
+        }
+      }
+      int issued = 0;
+      for (int idx = 0; idx < 2 * n_load; ++idx) {
+        const int sl = idx % kSlots;
+        if (!mbar_wait(bar_kvempty(sl), ((idx / kSlots) & 1) ^ 1, a.err, kErrWaitEmpty, abort_flag)) break;
+        const int k = kb + (idx >> 1);
+        const bool is_v = idx & 1;
+        const bool is_c = k < a.nC;
+        const int r0 = is_c ? k * 128 : (k - a.nC) * 128;
+        mbar_arrive_expect_tx(bar_kvfull(sl), L::kTileBytes);
+        const uint32_t dst = sb + L::kKV + sl * L::kTileBytes;
+        for (int at = 0; at < L::kAtoms; ++at) {
+          if (is_c) tma_load_4d(dst + at * L::kAtomBytes, is_v ? &tm_vc : &tm_kc, bar_kvfull(sl), at * 64, r0, g, s);
+          else tma_load_4d(dst + at * L::kAtomBytes, is_v ? &tm_vf : &tm_kf, bar_kvfull(sl), at * 64, g, r0, s);
+        }
+        issued = idx + 1;
+      }
+      if (nq) drain_wait(bar_q, 0, a.err);
+      for (int idx = (issued > kSlots ? issued - kSlots : 0); idx < issued; ++idx)
+        drain_wait(bar_kvfull(idx % kSlots), (idx / kSlots) & 1, a.err);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0 && n_load > 0) {
+      constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t id_o = idesc_bf16(128, D, false, true);
+      const int nX[2] = {nA, nB};
+      auto slot_addr = [&](int idx) { return sb + L::kKV + (idx % kSlots) * L::kTileBytes; };
+      auto wait_slot = [&](int idx) {
+        return mbar_wait(bar_kvfull(idx % kSlots), (idx / kSlots) & 1, a.err, kErrWaitLoad, abort_flag);
+      };
+      auto issue_s = [&](int x, int j) {  // S_x = Q_x K_j^T
+        const uint32_t qb = sb + L::kQ + x * L::kTileBytes, kbase = slot_addr(2 * j);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::kAtomBytes + (kk & 3) * 32;
+          mma_ss(tmem + col_s(x), sdesc_sw128(qb + off, 16, 1024), sdesc_sw128(kbase + off, 16, 1024), id_s,
+                 kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar_sfull(x));
+      };
+      auto issue_pv = [&](int x, int j) {  // O_x += P_x V_j
+        const uint32_t vbase = slot_addr(2 * j + 1);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + col_o(x), tmem + col_s(x) + kk * 8, sdesc_sw128(vbase + kk * 2048, L::kAtomBytes, 1024),
+                 id_o, (j > 0 || kk > 0) ? 1u : 0u);
+        if (j == nX[x] - 1) mma_commit(bar_odone(x));
+      };
+      bool ok = mbar_wait(bar_q, 0, a.err, kErrWaitLoad, abort_flag) && wait_slot(0);
+      if (ok) {
+        fence_after_sync();
+        if (nA > 0) issue_s(0, 0);
+        if (nB > 0) issue_s(1, 0);
+        mma_commit(bar_kvempty(0));
+      }
+      // Ring order of tiles: K_0, V_0, K_1, V_1, ...; each slot is released
+      // (kv_empty) after the last MMA reading it, in the same order.
+      for (int j = 0; ok && j < n_load; ++j) {
+        if (!(ok = wait_slot(2 * j + 1))) break;  // V_j
+        const bool next_k = j + 1 < n_load;
+        if (j < nA) {
+          if (!(ok = mbar_wait(bar_pfull(0), j & 1, a.err, kErrWaitP, abort_flag))) break;
+          fence_after_sync();
+          issue_pv(0, j);
+        }
+        if (next_k && !(ok = wait_slot(2 * (j + 1)))) break;  // K_{j+1}
+        if (j + 1 < nA) issue_s(0, j + 1);
+        if (j < nB) {
+          if (!(ok = mbar_wait(bar_pfull(1), j & 1, a.err, kErrWaitP, abort_flag))) break;
+          fence_after_sync();
+          issue_pv(1, j);
+        }
+        mma_commit(bar_kvempty((2 * j + 1) % kSlots));  // V_j read by both P.V
+        if (j + 1 < nB) issue_s(1, j + 1);
+        if (next_k) mma_commit(bar_kvempty((2 * (j + 1)) % kSlots));  // K_{j+1} read by both S
+      }
+      mma_commit(bar_done);
+      drain_wait(bar_done, 0, a.err);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax
+    const int x = (warp - 4) >> 2;  // 0: tile A, 1: tile B
+    const TileInfo ti = x == 0 ? tA : tB;
+    const int nX = x == 0 ? nA : nB;
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // row within the tile (= TMEM lane)
+    const int i = ti.i0 + r;            // query row in the frame
+    const uint32_t t_s = tmem + ((uint32_t)(quarter * 32) << 16) + col_s(x);
+    const uint32_t t_o = tmem + ((uint32_t)(quarter * 32) << 16) + col_o(x);
+    const float c = a.scale_log2;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = ti.valid;
+    for (int j = 0; ok && j < nX; ++j) {
+      if (!(ok = warp_wait(bar_sfull(x), j & 1, a.err, kErrWaitAcc, abort_flag))) break;
+      fence_after_sync();
+      const int k = kb + j;
+      const bool is_c = k < a.nC;
+      const int base = is_c ? k * 128 : (k - a.nC) * 128;
+      // visible columns of this row form a prefix [0, lim)
+      int lim = is_c ? a.m - base : (a.causal ? min(a.T, i + 1) : a.T) - base;
+      lim = max(0, min(128, lim));
+      const bool masked = __any_sync(0xffffffffu, lim < 128);
+      // pass 1: row max of the scaled logits
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c0 = 0; c0 < 4; ++c0) {
+        uint32_t v[32];
+        tmem_ld32(t_s + c0 * 32, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+          float sv = __uint_as_float(v[jj]) * c;
+          if (masked && c0 * 32 + jj >= lim) sv = -INFINITY;
+          mx = fmaxf(mx, sv);
+        }
+      }
+      float m_new = fmaxf(m_used, mx);
+      if (m_new == -INFINITY) m_new = 0.f;  // nothing visible yet in this row
+      if (j == 0) {
+        m_used = m_new;
+      } else {
+        const bool need = m_new > m_used + kRescaleLog2;
+        if (__any_sync(0xffffffffu, need)) {
+          // O holds P.V of earlier tiles, complete: S_j was issued after them
+          const float f = need ? ex2_approx(m_used - m_new) : 1.f;
+#pragma unroll
+          for (int c0 = 0; c0 < D / 32; ++c0) {
+            uint32_t v[32];
+            tmem_ld32(t_o + c0 * 32, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) v[jj] = __float_as_uint(__uint_as_float(v[jj]) * f);
+            tmem_st32(t_o + c0 * 32, v);
+          }
+          tmem_st_wait();
+          l *= f;
+          if (need) m_used = m_new;
+        }
+      }
+      // pass 2: P = exp2(S*c - m_used) as bf16 into the first 64 columns
+      float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+      for (int c0 = 0; c0 < 4; ++c0) {
+        uint32_t v[32];
+        tmem_ld32(t_s + c0 * 32, v);
+        tmem_ld_wait();
+        uint32_t pk[16];
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) {
+          float p0 = ex2_approx(fmaf(__uint_as_float(v[2 * jj]), c, -m_used));
+          float p1 = ex2_approx(fmaf(__uint_as_float(v[2 * jj + 1]), c, -m_used));
+          if (masked) {
+            if (c0 * 32 + 2 * jj >= lim) p0 = 0.f;
+            if (c0 * 32 + 2 * jj + 1 >= lim) p1 = 0.f;
+          }
+          ls0 += p0;
+          ls1 += p1;
+          pk[jj] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(t_s + c0 * 16, pk);
+      }
+      tmem_st_wait();
+      l += ls0 + ls1;
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_pfull(x));
+    }
+    // ---- epilogue: O / l and the row's log2-sum-exp
+    if (ok && nX > 0) ok = warp_wait(bar_odone(x), 0, a.err, kErrWaitAcc, abort_flag);
+    if (ok && ti.valid && !*abort_flag) {
+      fence_after_sync();
+      const bool row_ok = i < a.T;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float lse2 = l > 0.f ? m_used + __log2f(l) : -INFINITY;
+      if (a.n_split == 1) {
+        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + s * a.out_s + (long long)i * a.out_row +
+                              (long long)ti.h * D;
+#pragma unroll
+        for (int c0 = 0; c0 < D / 32; ++c0) {
+          uint32_t v[32];
+          tmem_ld32(t_o + c0 * 32, v);
+          tmem_ld_wait();
+          uint32_t pk[16];
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj)
+            pk[jj] = pack_bf16x2(__uint_as_float(v[2 * jj]) * inv, __uint_as_float(v[2 * jj + 1]) * inv);
+          if (row_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c0 * 32);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) dst[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+          }
+        }
+        if (row_ok && a.lse) a.lse[s * a.lse_s + (long long)ti.h * a.T + i] = lse2 * kLn2;
+      } else {
+        const long long prow = ((long long)(s * a.Hq + ti.h) * a.n_split + sp) * a.T + i;
+        float* orow = a.o_part + prow * D;
+#pragma unroll
+        for (int c0 = 0; c0 < D / 32; ++c0) {
+          uint32_t v[32];
+          if (nX > 0) {
+            tmem_ld32(t_o + c0 * 32, v);
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) v[jj] = 0u;
+          }
+          if (row_ok) {
+            float4* dst = reinterpret_cast<float4*>(orow + c0 * 32);
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4)
+              dst[q4] = make_float4(__uint_as_float(v[4 * q4]) * inv, __uint_as_float(v[4 * q4 + 1]) * inv,
+                                    __uint_as_float(v[4 * q4 + 2]) * inv, __uint_as_float(v[4 * q4 + 3]) * inv);
+          }
+        }
+        if (row_ok) a.ml_part[prow] = nX > 0 ? lse2 : -INFINITY;
+      }
+    }
+  }
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    fence_after_sync();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// Merge of key-split partials: one warp per query row.
+template <int D>
+__global__ void __launch_bounds__(256) attn_combine_kernel(AttnTcArgs a) {
+  const int warp_g = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  const int rows = a.S * a.Hq * a.T;
+  if (warp_g >= rows) return;
+  const int i = warp_g % a.T;
+  const int sh = warp_g / a.T;  // s * Hq + h
+  const int h = sh % a.Hq, s = sh / a.Hq;
+  const long long prow0 = (long long)sh * a.n_split * a.T + i;
+  float mx = -INFINITY;
+  for (int u = 0; u < a.n_split; ++u) mx = fmaxf(mx, a.ml_part[prow0 + (long long)u * a.T]);
+  constexpr int kPer = D / 32;
+  float acc[kPer];
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
+  float wsum = 0.f;
+  for (int u = 0; u < a.n_split; ++u) {
+    const float ml = a.ml_part[prow0 + (long long)u * a.T];
+    const float w = ml == -INFINITY ? 0.f : ex2_approx(ml - mx);
+    wsum += w;
+    const float* src = a.o_part + (prow0 + (long long)u * a.T) * D + lane * kPer;
+    if constexpr (kPer == 4) {
+      const float4 v = *reinterpret_cast<const float4*>(src);
+      acc[0] += w * v.x;
+      acc[1] += w * v.y;
+      acc[2] += w * v.z;
+      acc[3] += w * v.w;
+    } else {
+      const float2 v = *reinterpret_cast<const float2*>(src);
+      acc[0] += w * v.x;
+      acc[1] += w * v.y;
+    }
+  }
+  const float inv = 1.f / wsum;
+  __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + s * a.out_s + (long long)i * a.out_row +
+                        (long long)h * D + lane * kPer;
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) orow[e] = __float2bfloat16_rn(acc[e] * inv);
+  if (lane == 0 && a.lse) a.lse[s * a.lse_s + (long long)h * a.T + i] = (mx + __log2f(wsum)) * kLn2;
+}
+
+}  // namespace
+
+int attn_tc_splits(int S, int Hq, int Hkv, int T, int m, int n_sm) {
+  const int G = Hq / Hkv;
+  const int n_it = (T + 127) / 128;
+  const int n_pairs = (G * n_it + 1) / 2;
+  const int units = S * Hkv * n_pairs;
+  const int nk = (m + 127) / 128 + n_it;
+  int split = n_sm / units;
+  if (split < 1) split = 1;
+  if (split > nk) split = nk;
+  return split;
+}
+
+cudaError_t launch_attn_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kc, const CUtensorMap& tm_vc,
+                           const CUtensorMap& tm_kf, const CUtensorMap& tm_vf, const AttnTcArgs& a, int d,
+                           cudaStream_t st) {
+  const int units = a.S * a.Hkv * a.n_pairs * a.n_split;
+  cudaError_t e;
+  if (d == 128) {
+    const int smem = AttnSmem<128>::kAlloc;
+    if ((e = cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)))
+      return e;
+    attn_tc_kernel<128><<<units, kThreads, smem, st>>>(tm_q, tm_kc, tm_vc, tm_kf, tm_vf, a);
+  } else {
+    const int smem = AttnSmem<64>::kAlloc;
+    if ((e = cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)))
+      return e;
+    attn_tc_kernel<64><<<units, kThreads, smem, st>>>(tm_q, tm_kc, tm_vc, tm_kf, tm_vf, a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_combine(const AttnTcArgs& a, int d, cudaStream_t st) {
+  const long long rows = (long long)a.S * a.Hq * a.T;
+  const int blocks = (int)((rows * 32 + 255) / 256);
+  if (d == 128) attn_combine_kernel<128><<<blocks, 256, 0, st>>>(a);
+  else attn_combine_kernel<64><<<blocks, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace skv

@@ -37,6 +37,26 @@ struct ScoreTcArgs {
 cudaError_t launch_score_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kc, const CUtensorMap& tm_kf,
                             const ScoreTcArgs& a, int d, cudaStream_t st);
 
+// Tensor-core attention (bf16) over [compressed rows; frame tokens].
+struct AttnTcArgs {
+  void* out;          // out[s][i][h][dd] bf16
+  long long out_s;
+  int out_row;        // Hq * d
+  float* lse;         // [S][Hq][T] natural log, may be null
+  long long lse_s;
+  float* o_part;      // [S][Hq][n_split][T][d] f32 (n_split > 1)
+  float* ml_part;     // [S][Hq][n_split][T] log2-sum-exp
+  int m, T, Hq, Hkv, causal, S;
+  int n_it, n_pairs, n_split, nC, nF;
+  float scale_log2;
+  int* err;
+};
+int attn_tc_splits(int S, int Hq, int Hkv, int T, int m, int n_sm);
+cudaError_t launch_attn_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kc, const CUtensorMap& tm_vc,
+                           const CUtensorMap& tm_kf, const CUtensorMap& tm_vf, const AttnTcArgs& a, int d,
+                           cudaStream_t st);
+cudaError_t launch_attn_combine(const AttnTcArgs& a, int d, cudaStream_t st);
+
 // Message for statekv_last_error(NULL) (errors of calls without a handle).
 void set_free_error(const char* msg);
 

@@ -46,17 +46,6 @@ struct Smem {
   static constexpr int kAlloc = kBytes + 1024;            // room to align the base to 1024
 };
 
-// Bounded wait used on the teardown path only: ignores the abort flag.
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, int* err) {
-  const unsigned long long t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      atomicCAS(err, 0, kErrWaitDrain);
-      return;
-    }
-  }
-}
-
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kc,

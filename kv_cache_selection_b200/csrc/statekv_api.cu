@@ -14,6 +14,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <string>
 #include <vector>
@@ -54,6 +55,9 @@ struct statekv_handle {
   float* pool_score = nullptr;  // [S][Hkv][B+T]
   int32_t* idx = nullptr;       // [S][Hkv][max(B,1)]
   int* dev_err = nullptr;       // kernel error word (bounded-wait timeouts)
+  float* o_part = nullptr;      // attention key-split partials (bf16 path)
+  float* ml_part = nullptr;
+  int max_split = 1;
   // staging for statekv_prefill_frame_host (allocated on first use)
   void* stage_q = nullptr;
   void* stage_k = nullptr;
@@ -196,7 +200,8 @@ struct StageScope {
 
 // TMA maps of one step: q [S][T][Hq][d], K_C [S][Hkv][B][d], frame k [S][T][Hkv][d]
 int encode_step_maps(statekv_t h, const void* q, const void* kc, const void* k, CUtensorMap* tq,
-                     CUtensorMap* tkc, CUtensorMap* tkf) {
+                     CUtensorMap* tkc, CUtensorMap* tkf, const void* vc = nullptr, const void* v = nullptr,
+                     CUtensorMap* tvc = nullptr, CUtensorMap* tvf = nullptr) {
   const uint64_t d = h->d, Hq = h->Hq, Hkv = h->Hkv, T = h->T, S = h->S;
   const uint64_t B = std::max(h->B, 1);
   const uint64_t dq[4] = {d, Hq, T, S};
@@ -210,7 +215,9 @@ int encode_step_maps(statekv_t h, const void* q, const void* kc, const void* k, 
   int r;
   if ((r = skv::encode_tmap_bf16_4d(tq, q, dq, sq, bq)) != 0 ||
       (r = skv::encode_tmap_bf16_4d(tkc, kc, dc, sc, bc)) != 0 ||
-      (r = skv::encode_tmap_bf16_4d(tkf, k, dk, sk, bq)) != 0)
+      (r = skv::encode_tmap_bf16_4d(tkf, k, dk, sk, bq)) != 0 ||
+      (tvc && (r = skv::encode_tmap_bf16_4d(tvc, vc, dc, sc, bc)) != 0) ||
+      (tvf && (r = skv::encode_tmap_bf16_4d(tvf, v, dk, sk, bq)) != 0))
     return set_err(h, STATEKV_ERR_CUDA, "TMA tensor map encoding failed (CUresult %d)", r);
   return STATEKV_OK;
 }
@@ -224,6 +231,97 @@ int launch_err(statekv_t h, cudaError_t e, const char* what) {
 namespace skv {
 void set_free_error(const char* msg) { g_free_error = msg; }
 }  // namespace skv
+
+namespace {
+
+// Process-wide scratch of full_causal_prefill's key-split partials, grown on
+// demand (one buffer per device, guarded by a mutex).
+std::mutex g_fc_mu;
+struct FcScratch {
+  float* o = nullptr;
+  float* ml = nullptr;
+  int* err = nullptr;
+  size_t o_bytes = 0, ml_bytes = 0;
+};
+FcScratch g_fc[64];
+
+int full_causal_tc(const void* q, const void* k, const void* v, int n_seq, int N, int Hq, int Hkv, int d,
+                   void* out, float* lse, cudaStream_t st) {
+  int dev = 0, n_sm = 148;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= 64)
+    return set_err(nullptr, STATEKV_ERR_CUDA, "no usable CUDA device");
+  cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+  skv::AttnTcArgs ta{};
+  ta.out = out;
+  ta.out_s = (long long)N * Hq * d;
+  ta.out_row = Hq * d;
+  ta.lse = lse;
+  ta.lse_s = (long long)Hq * N;
+  ta.m = 0;
+  ta.T = N;
+  ta.Hq = Hq;
+  ta.Hkv = Hkv;
+  ta.causal = 1;
+  ta.S = n_seq;
+  ta.n_it = (N + 127) / 128;
+  ta.n_pairs = ((Hq / Hkv) * ta.n_it + 1) / 2;
+  ta.n_split = skv::attn_tc_splits(n_seq, Hq, Hkv, N, 0, n_sm);
+  ta.nC = 0;
+  ta.nF = ta.n_it;
+  ta.scale_log2 = skv::kLog2e / sqrtf((float)d);
+  {
+    std::lock_guard<std::mutex> lk(g_fc_mu);
+    FcScratch& sc = g_fc[dev];
+    const size_t ob = ta.n_split > 1 ? (size_t)n_seq * Hq * ta.n_split * N * d * 4 : 16;
+    const size_t mb = ta.n_split > 1 ? (size_t)n_seq * Hq * ta.n_split * N * 4 : 16;
+    if (!sc.err && cudaMalloc((void**)&sc.err, 16) == cudaSuccess) cudaMemset(sc.err, 0, 16);
+    if (sc.o_bytes < ob) {
+      if (sc.o) cudaFree(sc.o);
+      sc.o = nullptr;
+      sc.o_bytes = 0;
+      if (cudaMalloc((void**)&sc.o, ob) != cudaSuccess) {
+        cudaGetLastError();
+        return set_err(nullptr, STATEKV_ERR_OOM, "scratch allocation of %zu bytes failed", ob);
+      }
+      sc.o_bytes = ob;
+    }
+    if (sc.ml_bytes < mb) {
+      if (sc.ml) cudaFree(sc.ml);
+      sc.ml = nullptr;
+      sc.ml_bytes = 0;
+      if (cudaMalloc((void**)&sc.ml, mb) != cudaSuccess) {
+        cudaGetLastError();
+        return set_err(nullptr, STATEKV_ERR_OOM, "scratch allocation of %zu bytes failed", mb);
+      }
+      sc.ml_bytes = mb;
+    }
+    if (!sc.err) return set_err(nullptr, STATEKV_ERR_OOM, "error-word allocation failed");
+    ta.o_part = sc.o;
+    ta.ml_part = sc.ml;
+    ta.err = sc.err;
+  }
+  // q [S][N][Hq][d] and k, v [S][N][Hkv][d]: the whole sequence is the "frame"
+  const uint64_t D = d;
+  const uint64_t dq[4] = {D, (uint64_t)Hq, (uint64_t)N, (uint64_t)n_seq};
+  const uint64_t sq[3] = {D * 2, (uint64_t)Hq * D * 2, (uint64_t)N * Hq * D * 2};
+  const uint64_t dk[4] = {D, (uint64_t)Hkv, (uint64_t)N, (uint64_t)n_seq};
+  const uint64_t sk[3] = {D * 2, (uint64_t)Hkv * D * 2, (uint64_t)N * Hkv * D * 2};
+  const uint32_t box[4] = {64, 1, 128, 1};
+  CUtensorMap tq, tk, tv;
+  int r;
+  if ((r = skv::encode_tmap_bf16_4d(&tq, q, dq, sq, box)) || (r = skv::encode_tmap_bf16_4d(&tk, k, dk, sk, box)) ||
+      (r = skv::encode_tmap_bf16_4d(&tv, v, dk, sk, box)))
+    return set_err(nullptr, STATEKV_ERR_CUDA, "TMA tensor map encoding failed (CUresult %d)", r);
+  // no compressed rows: the C maps are never read
+  if ((e = skv::launch_attn_tc(tq, tk, tv, tk, tv, ta, d, st)) != cudaSuccess)
+    return set_err(nullptr, STATEKV_ERR_CUDA, "attention launch failed: %s", cudaGetErrorString(e));
+  if (ta.n_split > 1 && (e = skv::launch_attn_combine(ta, d, st)) != cudaSuccess)
+    return set_err(nullptr, STATEKV_ERR_CUDA, "attention combine launch failed: %s", cudaGetErrorString(e));
+  return STATEKV_OK;
+}
+
+}  // namespace
 
 extern "C" {
 
@@ -261,6 +359,16 @@ int statekv_create_batched(statekv_t* out, int n_streams, int Hq, int Hkv, int d
     g_free_error = h->err;
     statekv_destroy(h);
     return rc;
+  }
+  if (dtype == STATEKV_BF16) {
+    h->max_split = skv::attn_tc_splits(n_streams, Hq, Hkv, T, B, h->n_sm);
+    if (h->max_split > 1 &&
+        ((rc = dev_alloc(h, (void**)&h->o_part, (size_t)n_streams * Hq * h->max_split * T * d * 4)) ||
+         (rc = dev_alloc(h, (void**)&h->ml_part, (size_t)n_streams * Hq * h->max_split * T * 4)))) {
+      g_free_error = h->err;
+      statekv_destroy(h);
+      return rc;
+    }
   }
   *out = h;
   return STATEKV_OK;
@@ -327,7 +435,42 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
   aa.Hkv = Hkv;
   aa.causal = h->mask == STATEKV_MASK_FRAME_CAUSAL;
   aa.scale_log2 = scale_log2;
-  {
+  CUtensorMap tq, tkc, tkf, tvc, tvf;
+  if (h->dtype == STATEKV_BF16) {
+    if ((rc = encode_step_maps(h, q, L->kc[cur], k, &tq, &tkc, &tkf, L->vc[cur], v, &tvc, &tvf))) return rc;
+    skv::AttnTcArgs ta{};
+    ta.out = out;
+    ta.out_s = (long long)T * Hq * d;
+    ta.out_row = Hq * d;
+    ta.lse = h->lse;
+    ta.lse_s = (long long)Hq * T;
+    ta.o_part = h->o_part;
+    ta.ml_part = h->ml_part;
+    ta.m = m;
+    ta.T = T;
+    ta.Hq = Hq;
+    ta.Hkv = Hkv;
+    ta.causal = aa.causal;
+    ta.S = S;
+    ta.n_it = (T + 127) / 128;
+    ta.n_pairs = ((Hq / Hkv) * ta.n_it + 1) / 2;
+    ta.n_split = std::min(h->max_split, skv::attn_tc_splits(S, Hq, Hkv, T, m, h->n_sm));
+    ta.nC = (m + 127) / 128;
+    ta.nF = ta.n_it;
+    ta.scale_log2 = scale_log2;
+    ta.err = h->dev_err;
+    {
+      StageScope sc(h, st, STATEKV_STAGE_ATTENTION);
+      if ((e = skv::launch_attn_tc(tq, tkc, tvc, tkf, tvf, ta, d, st)) != cudaSuccess)
+        return launch_err(h, e, "attention");
+      sc.done();
+    }
+    if (ta.n_split > 1) {
+      StageScope sc(h, st, STATEKV_STAGE_ATTENTION_COMBINE);
+      if ((e = skv::launch_attn_combine(ta, d, st)) != cudaSuccess) return launch_err(h, e, "attention combine");
+      sc.done();
+    }
+  } else {
     StageScope sc(h, st, STATEKV_STAGE_ATTENTION);
     if ((e = skv::launch_attn_simt(aa, h->dtype, d, S, st)) != cudaSuccess) return launch_err(h, e, "attention");
     sc.done();
@@ -357,8 +500,6 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
   sa.causal = aa.causal;
   sa.scale_log2 = scale_log2;
   if (h->dtype == STATEKV_BF16) {
-    CUtensorMap tq, tkc, tkf;
-    if ((rc = encode_step_maps(h, q, L->kc[cur], k, &tq, &tkc, &tkf))) return rc;
     skv::ScoreTcArgs ta{};
     ta.lse = h->lse;
     ta.lse_s = aa.lse_s;
@@ -588,6 +729,10 @@ int full_causal_prefill_batched(const void* q, const void* k, const void* v, int
     return set_err(nullptr, STATEKV_ERR_INVALID_ARG, "bad dtype %d", dtype);
   if (d != 64 && d != 128) return set_err(nullptr, STATEKV_ERR_UNSUPPORTED, "head dim %d", d);
   if (n_tokens == 0) return STATEKV_OK;
+  if (((uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)out) & 15)
+    return set_err(nullptr, STATEKV_ERR_INVALID_ARG, "q/k/v/out must be 16-byte aligned");
+  if (dtype == STATEKV_BF16) return full_causal_tc(q, k, v, n_seq, n_tokens, Hq, Hkv, d, out, lse,
+                                                   static_cast<cudaStream_t>(stream));
   skv::AttnArgs aa{};
   aa.q = q;
   aa.q_s = (long long)n_tokens * Hq * d;
