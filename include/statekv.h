@@ -139,8 +139,8 @@ int statekv_get_detailed(statekv_t h, int layer, const void** k, const void** v,
 /* Borrow the per-row statistics of the most recent prefill_frame (any layer):
  *   lse        [S][Hq][T] float32, natural-log log-sum-exp of each query row;
  *   pool_score [S][Hkv][B+T] float32, the score of every pool candidate
- *              (C entries first, then frame tokens; rows identical in GLOBAL
- *              mode); entries [0, pool_len) valid.
+ *              (C entries first, then frame tokens); entries [0, pool_len)
+ *              valid.  In GLOBAL mode only row 0 of each stream is written.
  * Valid until the next prefill_frame.  Any output pointer may be NULL. */
 int statekv_get_step_stats(statekv_t h, const float** lse, const float** pool_score,
                            int* pool_len);

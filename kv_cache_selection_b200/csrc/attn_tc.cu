@@ -29,6 +29,7 @@
 #include "kernels.h"
 #include "tc_common.cuh"
 
+
 namespace skv {
 namespace {
 using namespace tc;
@@ -135,6 +136,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
   // TMEM columns: S/P of tile A at 0, of tile B at 128, O of A at 256, O of B at 384
   auto col_s = [](int x) { return (uint32_t)(x * 128); };
   auto col_o = [](int x) { return (uint32_t)(256 + x * 128); };
@@ -349,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (row_ok && a.lse) a.lse[s * a.lse_s + (long long)ti.h * a.T + i] = lse2 * kLn2;
       } else {
         const long long prow = ((long long)(s * a.Hq + ti.h) * a.n_split + sp) * a.T + i;
-        float* orow = a.o_part + prow * D;
+        __nv_bfloat16* orow = a.o_part + prow * D;
 #pragma unroll
         for (int c0 = 0; c0 < D / 32; ++c0) {
           uint32_t v[32];
@@ -360,12 +363,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj) v[jj] = 0u;
           }
-          if (row_ok) {
-            float4* dst = reinterpret_cast<float4*>(orow + c0 * 32);
+          uint32_t pk[16];
 #pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4)
-              dst[q4] = make_float4(__uint_as_float(v[4 * q4]) * inv, __uint_as_float(v[4 * q4 + 1]) * inv,
-                                    __uint_as_float(v[4 * q4 + 2]) * inv, __uint_as_float(v[4 * q4 + 3]) * inv);
+          for (int jj = 0; jj < 16; ++jj)
+            pk[jj] = pack_bf16x2(__uint_as_float(v[2 * jj]) * inv, __uint_as_float(v[2 * jj + 1]) * inv);
+          if (row_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c0 * 32);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) dst[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
           }
         }
         if (row_ok) a.ml_part[prow] = nX > 0 ? lse2 : -INFINITY;
@@ -380,46 +385,60 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Merge of key-split partials: one warp per query row.
+// Merge of key-split partials.  One thread per (query row, 8-element chunk of
+// d): it reads the row's n_split log2-sum-exps and its chunk of every split's
+// O/l at once (independent loads), weights them by 2^(ml_u - max) and writes
+// the bf16 result; chunk 0 also writes the row's natural-log lse.
+constexpr int kMaxSplit = 8;
+
 template <int D>
 __global__ void __launch_bounds__(256) attn_combine_kernel(AttnTcArgs a) {
-  const int warp_g = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_trigger();
+  constexpr int kChunks = D / 8;
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
   const int rows = a.S * a.Hq * a.T;
-  if (warp_g >= rows) return;
-  const int i = warp_g % a.T;
-  const int sh = warp_g / a.T;  // s * Hq + h
+  if (t >= rows * kChunks) return;
+  const int chunk = t % kChunks;
+  const int rw = t / kChunks;
+  const int i = rw % a.T;
+  const int sh = rw / a.T;  // s * Hq + h
   const int h = sh % a.Hq, s = sh / a.Hq;
   const long long prow0 = (long long)sh * a.n_split * a.T + i;
-  float mx = -INFINITY;
-  for (int u = 0; u < a.n_split; ++u) mx = fmaxf(mx, a.ml_part[prow0 + (long long)u * a.T]);
-  constexpr int kPer = D / 32;
-  float acc[kPer];
+  float ml[kMaxSplit];
+  uint4 raw[kMaxSplit];
 #pragma unroll
-  for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
+  for (int u = 0; u < kMaxSplit; ++u) {
+    if (u < a.n_split) {
+      ml[u] = __ldg(a.ml_part + prow0 + (long long)u * a.T);
+      raw[u] = __ldg(reinterpret_cast<const uint4*>(a.o_part + (prow0 + (long long)u * a.T) * D) + chunk);
+    }
+  }
+  float mx = -INFINITY;
+#pragma unroll
+  for (int u = 0; u < kMaxSplit; ++u)
+    if (u < a.n_split) mx = fmaxf(mx, ml[u]);
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   float wsum = 0.f;
-  for (int u = 0; u < a.n_split; ++u) {
-    const float ml = a.ml_part[prow0 + (long long)u * a.T];
-    const float w = ml == -INFINITY ? 0.f : ex2_approx(ml - mx);
-    wsum += w;
-    const float* src = a.o_part + (prow0 + (long long)u * a.T) * D + lane * kPer;
-    if constexpr (kPer == 4) {
-      const float4 v = *reinterpret_cast<const float4*>(src);
-      acc[0] += w * v.x;
-      acc[1] += w * v.y;
-      acc[2] += w * v.z;
-      acc[3] += w * v.w;
-    } else {
-      const float2 v = *reinterpret_cast<const float2*>(src);
-      acc[0] += w * v.x;
-      acc[1] += w * v.y;
+#pragma unroll
+  for (int u = 0; u < kMaxSplit; ++u) {
+    if (u < a.n_split) {
+      const float w = ml[u] == -INFINITY ? 0.f : ex2_approx(ml[u] - mx);
+      wsum += w;
+      const __nv_bfloat16* v = reinterpret_cast<const __nv_bfloat16*>(&raw[u]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += w * __bfloat162float(v[e]);
     }
   }
   const float inv = 1.f / wsum;
-  __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + s * a.out_s + (long long)i * a.out_row +
-                        (long long)h * D + lane * kPer;
+  uint4 o;
+  uint32_t* op = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
-  for (int e = 0; e < kPer; ++e) orow[e] = __float2bfloat16_rn(acc[e] * inv);
-  if (lane == 0 && a.lse) a.lse[s * a.lse_s + (long long)h * a.T + i] = (mx + __log2f(wsum)) * kLn2;
+  for (int e = 0; e < 4; ++e) op[e] = pack_bf16x2(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+  __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + s * a.out_s + (long long)i * a.out_row +
+                        (long long)h * D;
+  reinterpret_cast<uint4*>(orow)[chunk] = o;
+  if (chunk == 0 && a.lse) a.lse[s * a.lse_s + (long long)h * a.T + i] = (mx + __log2f(wsum)) * kLn2;
 }
 
 }  // namespace
@@ -433,34 +452,36 @@ int attn_tc_splits(int S, int Hq, int Hkv, int T, int m, int n_sm) {
   int split = n_sm / units;
   if (split < 1) split = 1;
   if (split > nk) split = nk;
+  if (split > kMaxSplit) split = kMaxSplit;
   return split;
 }
 
 cudaError_t launch_attn_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kc, const CUtensorMap& tm_vc,
                            const CUtensorMap& tm_kf, const CUtensorMap& tm_vf, const AttnTcArgs& a, int d,
-                           cudaStream_t st) {
+                           cudaStream_t st, bool pdl) {
   const int units = a.S * a.Hkv * a.n_pairs * a.n_split;
   cudaError_t e;
   if (d == 128) {
     const int smem = AttnSmem<128>::kAlloc;
     if ((e = cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)))
       return e;
-    attn_tc_kernel<128><<<units, kThreads, smem, st>>>(tm_q, tm_kc, tm_vc, tm_kf, tm_vf, a);
+    return launch_kernel(attn_tc_kernel<128>, dim3(units), dim3(kThreads), smem, st, pdl, tm_q, tm_kc, tm_vc,
+                         tm_kf, tm_vf, a);
   } else {
     const int smem = AttnSmem<64>::kAlloc;
     if ((e = cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)))
       return e;
-    attn_tc_kernel<64><<<units, kThreads, smem, st>>>(tm_q, tm_kc, tm_vc, tm_kf, tm_vf, a);
+    return launch_kernel(attn_tc_kernel<64>, dim3(units), dim3(kThreads), smem, st, pdl, tm_q, tm_kc, tm_vc,
+                         tm_kf, tm_vf, a);
   }
   return cudaGetLastError();
 }
 
-cudaError_t launch_attn_combine(const AttnTcArgs& a, int d, cudaStream_t st) {
+cudaError_t launch_attn_combine(const AttnTcArgs& a, int d, cudaStream_t st, bool pdl) {
   const long long rows = (long long)a.S * a.Hq * a.T;
-  const int blocks = (int)((rows * 32 + 255) / 256);
-  if (d == 128) attn_combine_kernel<128><<<blocks, 256, 0, st>>>(a);
-  else attn_combine_kernel<64><<<blocks, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  const int blocks = (int)((rows * (d / 8) + 255) / 256);
+  if (d == 128) return launch_kernel(attn_combine_kernel<128>, dim3(blocks), dim3(256), 0, st, pdl, a);
+  return launch_kernel(attn_combine_kernel<64>, dim3(blocks), dim3(256), 0, st, pdl, a);
 }
 
 }  // namespace skv

@@ -10,6 +10,12 @@ namespace skv {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
+// Programmatic dependent launch: wait until the preceding kernel in the stream
+// has completed and its writes are visible (a no-op without a programmatic
+// dependency), and let the next kernel start its prologue early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
 
@@ -76,12 +82,10 @@ struct SelectArgs {
   const float* part;      // part[s][g][j], j < m + T
   long long part_s;
   int part_g;
-  float* pool_score;      // out, same layout as part
+  float* pool_score;      // out, same layout as part (row of the selection group only)
   const int32_t* pos_c;   // current C positions [s][g][B]
   const int32_t* pos_f;   // frame positions [s][T]
-  int32_t* idx;           // out [s][g][B] kept pool indices, ascending
-  int32_t* pos_new;       // out [s][g][B]
-  float* score_new;       // out [s][g][B]
+  int32_t* idx;           // out [s][g][B] kept pool indices, ascending (row 0 in global mode)
   int Hkv, m, T, B, global;
 };
 
@@ -95,6 +99,11 @@ struct GatherArgs {
   void* kd;        void* vd;         // D [s][g][max_tok][d]
   int32_t* pos_d;                    // [s][max_tok]
   const int32_t* pos_f;              // [s][T]
+  const int32_t* pos_c;              // current C positions [s][g][B]
+  const float* pool_score;           // [s][g][pool_g] (row 0 only in global mode)
+  int32_t* pos_new;                  // next C positions [s][g][B]
+  float* score_new;                  // next C scores [s][g][B]
+  int pool_g;                        // row stride of pool_score
   int Hkv, T, B, m, m_new, row_bytes, global, d_len, max_tok;
   int S;
 };

@@ -8,13 +8,31 @@
 
 namespace skv {
 
+// Launch with an optional programmatic stream serialisation attribute (the
+// kernel must call pdl_wait() before reading its predecessor's output).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                          bool pdl, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 constexpr int kDtypeBF16 = 0;
 constexpr int kDtypeF32 = 1;
 
 cudaError_t launch_attn_simt(const AttnArgs& a, int dtype, int d, int S, cudaStream_t st);
 cudaError_t launch_score_simt(const ScoreArgs& a, int dtype, int d, int S, cudaStream_t st);
-cudaError_t launch_select(const SelectArgs& a, int S, cudaStream_t st);
-cudaError_t launch_gather(const GatherArgs& a, int n_sm, cudaStream_t st);
+cudaError_t launch_select(const SelectArgs& a, int S, cudaStream_t st, bool pdl = false);
+cudaError_t launch_gather(const GatherArgs& a, int n_sm, cudaStream_t st, bool pdl = false);
 
 // bf16 4-D tiled TMA map, 128-byte swizzle, zero fill out of bounds.  dims[0]
 // is the innermost (contiguous) extent in elements; strides_bytes[i] is the
@@ -35,7 +53,7 @@ struct ScoreTcArgs {
   int* err;          // device error word (timeouts)
 };
 cudaError_t launch_score_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kc, const CUtensorMap& tm_kf,
-                            const ScoreTcArgs& a, int d, cudaStream_t st);
+                            const ScoreTcArgs& a, int d, cudaStream_t st, bool pdl = false);
 
 // Tensor-core attention (bf16) over [compressed rows; frame tokens].
 struct AttnTcArgs {
@@ -44,7 +62,7 @@ struct AttnTcArgs {
   int out_row;        // Hq * d
   float* lse;         // [S][Hq][T] natural log, may be null
   long long lse_s;
-  float* o_part;      // [S][Hq][n_split][T][d] f32 (n_split > 1)
+  __nv_bfloat16* o_part;  // [S][Hq][n_split][T][d] O/l per split (n_split > 1)
   float* ml_part;     // [S][Hq][n_split][T] log2-sum-exp
   int m, T, Hq, Hkv, causal, S;
   int n_it, n_pairs, n_split, nC, nF;
@@ -54,8 +72,8 @@ struct AttnTcArgs {
 int attn_tc_splits(int S, int Hq, int Hkv, int T, int m, int n_sm);
 cudaError_t launch_attn_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kc, const CUtensorMap& tm_vc,
                            const CUtensorMap& tm_kf, const CUtensorMap& tm_vf, const AttnTcArgs& a, int d,
-                           cudaStream_t st);
-cudaError_t launch_attn_combine(const AttnTcArgs& a, int d, cudaStream_t st);
+                           cudaStream_t st, bool pdl = false);
+cudaError_t launch_attn_combine(const AttnTcArgs& a, int d, cudaStream_t st, bool pdl = false);
 
 // Message for statekv_last_error(NULL) (errors of calls without a handle).
 void set_free_error(const char* msg);

@@ -35,15 +35,14 @@ struct Smem {
   static constexpr int kTileBytes = kAtoms * kAtomBytes;
   static constexpr int kK = 0;
   static constexpr int kQ = kK + kTileBytes;
-  static constexpr int kLse = kQ + kStages * kTileBytes;  // per epilogue warp: 64 floats
-  static constexpr int kRed = kLse + kEpiWarps * 64 * 4;  // 128 floats
+  static constexpr int kRed = kQ + kStages * kTileBytes;  // 128 floats
   static constexpr int kBar = kRed + 128 * 4;
   // k_full, q_full[kStages], q_empty[kStages], acc_full[2], acc_empty[2], done
   static constexpr int kNumBars = 1 + 2 * kStages + 4 + 1;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
-  static constexpr int kBytes = kAbort + 4;
-  static constexpr int kAlloc = kBytes + 1024;            // room to align the base to 1024
+  static constexpr int kLse = (kAbort + 4 + 15) & ~15;    // [G][n_ic*128] row statistics follow
+  static constexpr int kAlloc = kLse + 1024;              // + room to align the base to 1024
 };
 
 template <int D>
@@ -97,6 +96,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -154,22 +155,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int half = ew >> 2;             // which 64 columns of each chunk
     const int row = quarter * 32 + lane;  // key row within the tile
     const int key = r0 + row;
-    float* lse2 = reinterpret_cast<float*>(smem + L::kLse) + ew * 64;
+    // row statistics of the whole group in log2 units, +inf past the frame
+    const int tpad = n_ic * 128;
+    float* lse_all = reinterpret_cast<float*>(smem + L::kLse);
+    for (int e = threadIdx.x - 64; e < G * tpad; e += 32 * kEpiWarps) {
+      const int hh = e / tpad, i = e % tpad;
+      lse_all[e] = i < a.T ? a.lse[s * a.lse_s + (long long)(g * G + hh) * a.T + i] * kLog2e : INFINITY;
+    }
+    named_bar_sync(2, 32 * kEpiWarps);
     float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
     bool ok = true;
     for (int c = 0; c < n_chunks; ++c) {
       const int buf = c & 1;
-      const int h = g * G + c / per_head;
+      const int hh = c / per_head;
       const int i0 = (ic_min + c % per_head) * 128;
       const int cbase = i0 + half * 64;
-      // this warp's 64 row statistics, in log2 units (+inf past the frame)
-      __syncwarp();
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int i = cbase + lane + 32 * u;
-        lse2[lane + 32 * u] = i < a.T ? a.lse[s * a.lse_s + (long long)h * a.T + i] * kLog2e : INFINITY;
-      }
-      __syncwarp();
+      const float* lse2 = lse_all + hh * tpad + cbase;
       uint32_t got = 1;
       if (lane == 0) got = mbar_wait(bar_accfull(buf), (c >> 1) & 1, a.err, kErrWaitAcc, abort_flag) ? 1u : 0u;
       got = __shfl_sync(0xffffffffu, got, 0);
@@ -180,11 +181,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_after_sync();
       // some of this warp's columns precede some key of the tile (warp-uniform)
       const bool diag = !is_c && a.causal && (cbase < r0 + 127);
+      uint32_t rr[2][32];
+      tmem_ld32(tmem_addr(tmem, quarter * 32, buf * 128 + half * 64), rr[0]);
+      tmem_ld32(tmem_addr(tmem, quarter * 32, buf * 128 + half * 64 + 32), rr[1]);
+      tmem_ld_wait();
 #pragma unroll
       for (int q32 = 0; q32 < 2; ++q32) {
-        uint32_t r[32];
-        tmem_ld32(tmem_addr(tmem, quarter * 32, buf * 128 + half * 64 + q32 * 32), r);
-        tmem_ld_wait();
+        const uint32_t* r = rr[q32];
         const float4* l4 = reinterpret_cast<const float4*>(lse2 + q32 * 32);
 #pragma unroll
         for (int j4 = 0; j4 < 8; ++j4) {
@@ -235,21 +238,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 cudaError_t launch_score_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kc, const CUtensorMap& tm_kf,
-                            const ScoreTcArgs& a, int d, cudaStream_t st) {
+                            const ScoreTcArgs& a, int d, cudaStream_t st, bool pdl) {
   const int n_tiles = a.n_c_tiles + a.n_f_tiles;
   if (n_tiles == 0) return cudaSuccess;
   dim3 grid(n_tiles, a.Hkv, a.S);
   cudaError_t e;
+  const int n_ic = (a.T + 127) / 128;
+  const int lse_bytes = (a.Hq / a.Hkv) * n_ic * 128 * 4;
   if (d == 128) {
-    const int smem = Smem<128>::kAlloc;
+    const int smem = Smem<128>::kAlloc + lse_bytes;
     if ((e = cudaFuncSetAttribute(score_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)))
       return e;
-    score_tc_kernel<128><<<grid, kThreads, smem, st>>>(tm_q, tm_kc, tm_kf, a);
+    return launch_kernel(score_tc_kernel<128>, grid, dim3(kThreads), smem, st, pdl, tm_q, tm_kc, tm_kf, a);
   } else {
-    const int smem = Smem<64>::kAlloc;
+    const int smem = Smem<64>::kAlloc + lse_bytes;
     if ((e = cudaFuncSetAttribute(score_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)))
       return e;
-    score_tc_kernel<64><<<grid, kThreads, smem, st>>>(tm_q, tm_kc, tm_kf, a);
+    return launch_kernel(score_tc_kernel<64>, grid, dim3(kThreads), smem, st, pdl, tm_q, tm_kc, tm_kf, a);
   }
   return cudaGetLastError();
 }

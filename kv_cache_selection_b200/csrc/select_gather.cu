@@ -17,6 +17,7 @@ namespace skv {
 namespace {
 
 constexpr int kSelThreads = 1024;
+constexpr int kSelWarps = kSelThreads / 32;
 
 __device__ __forceinline__ uint32_t score_bits(float x) {
   // scores are sums of exponentials: >= +0, so the IEEE bit pattern orders
@@ -24,7 +25,7 @@ __device__ __forceinline__ uint32_t score_bits(float x) {
   return __float_as_uint(x);
 }
 
-// Block-wide exclusive scan of one 32-bit value per thread (1024 threads).
+// Block-wide exclusive scan of one 32-bit value per thread.
 __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* warp_tot) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t incl = v;
@@ -36,14 +37,14 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* w
   if (lane == 31) warp_tot[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    uint32_t w = warp_tot[lane];
+    uint32_t w = lane < kSelWarps ? warp_tot[lane] : 0u;
     uint32_t wi = w;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
       uint32_t n = __shfl_up_sync(0xffffffffu, wi, off);
       if (lane >= off) wi += n;
     }
-    warp_tot[lane] = wi - w;  // exclusive
+    if (lane < kSelWarps) warp_tot[lane] = wi - w;  // exclusive
   }
   __syncthreads();
   uint32_t r = warp_tot[warp] + incl - v;
@@ -52,185 +53,242 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* w
 }
 
 // One block per (selection group, stream).  Dynamic shared memory holds the
-// pool's scores (L floats).
+// pool's scores (L floats).  Radix select on 8-bit digits, most significant
+// first; each pass is a histogram (warp-aggregated shared atomics) and a
+// suffix count over the 256 bins done with warp shuffles.
 __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) {
   extern __shared__ float sc[];
   __shared__ uint32_t hist[257];
-  __shared__ uint32_t suffix[257];
+  __shared__ uint32_t bin_tot[8];
   __shared__ uint32_t warp_tot[32];
-  __shared__ uint32_t sel_bin;
+  __shared__ uint32_t sel_bin, sel_above;
   const int grp = blockIdx.x, s = blockIdx.y;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int L = a.m + a.T;
   const int G0 = a.global ? 0 : grp;
   const int G1 = a.global ? a.Hkv : grp + 1;
+  pdl_wait();
+  pdl_trigger();
 
-  // 1. scores of the pool: global mode sums the KV groups in a fixed order
-  for (int j = threadIdx.x; j < L; j += kSelThreads) {
-    float v = 0.f;
-    for (int g = G0; g < G1; ++g) v += a.part[s * a.part_s + (long long)g * a.part_g + j];
-    sc[j] = v;
-    for (int g = G0; g < G1; ++g) a.pool_score[s * a.part_s + (long long)g * a.part_g + j] = v;
+  // 1. scores of the pool (global mode sums the KV groups in a fixed order)
+  //    and the pool positions, staged in shared memory; every load of a
+  //    candidate is independent of the others
+  int* posp = reinterpret_cast<int*>(sc + L);
+  const float* __restrict__ part = a.part + s * a.part_s;
+  const int* __restrict__ pos_c = a.pos_c + ((long long)s * a.Hkv + G0) * a.B;
+  const int* __restrict__ pos_f = a.pos_f + (long long)s * a.T;
+  constexpr int kBatch = 4;  // candidates per thread whose loads are in flight together
+  for (int jb = 0; jb < L; jb += kBatch * kSelThreads) {
+    float pv[kBatch][8];
+    int pp[kBatch];
+#pragma unroll
+    for (int q = 0; q < kBatch; ++q) {
+      const int j = jb + q * kSelThreads + threadIdx.x;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        pv[q][u] = (j < L && G0 + u < G1) ? __ldg(part + (long long)(G0 + u) * a.part_g + j) : 0.f;
+      pp[q] = j < L ? (j < a.m ? __ldg(pos_c + j) : __ldg(pos_f + (j - a.m))) : 0;
+    }
+#pragma unroll
+    for (int q = 0; q < kBatch; ++q) {
+      const int j = jb + q * kSelThreads + threadIdx.x;
+      if (j < L) {
+        float v = 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v += pv[q][u];
+        sc[j] = v;
+        posp[j] = pp[q];
+      }
+    }
   }
+  for (int b = threadIdx.x; b < 257; b += kSelThreads) hist[b] = 0;
   __syncthreads();
+  for (int j = threadIdx.x; j < L; j += kSelThreads) a.pool_score[s * a.part_s + (long long)G0 * a.part_g + j] = sc[j];
   if (a.B <= 0) return;  // nothing is kept (block-uniform)
 
-  // 2. threshold: the B-th largest score (radix select, 8 bits per pass)
+  // 2. threshold: the B-th largest score
   uint32_t tau = 0;
   int need_eq = 0;  // how many candidates equal to tau are kept
   const bool keep_all = L <= a.B;
   if (!keep_all) {
     uint32_t prefix = 0, pmask = 0;
     int k = a.B;
+    const int n_iter = (L + kSelThreads - 1) / kSelThreads;
     for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int b = threadIdx.x; b < 257; b += kSelThreads) hist[b] = 0;
-      __syncthreads();
-      const int n_iter = (L + kSelThreads - 1) / kSelThreads;
       for (int it = 0; it < n_iter; ++it) {
         const int j = it * kSelThreads + threadIdx.x;
         uint32_t digit = 256;
         if (j < L) {
-          uint32_t u = score_bits(sc[j]);
+          const uint32_t u = score_bits(sc[j]);
           if ((u & pmask) == prefix) digit = (u >> shift) & 255u;
         }
         const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-        if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
+        if (lane == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
       }
       __syncthreads();
-      // suffix[b] = number of candidates (matching the prefix) with digit >= b
-      if (threadIdx.x < 256) suffix[threadIdx.x] = hist[threadIdx.x];
-      if (threadIdx.x == 0) suffix[256] = 0;
-      __syncthreads();
-      for (int off = 1; off < 256; off <<= 1) {
-        uint32_t add = 0;
-        if (threadIdx.x < 256 && threadIdx.x + off < 256) add = suffix[threadIdx.x + off];
-        __syncthreads();
-        if (threadIdx.x < 256) suffix[threadIdx.x] += add;
-        __syncthreads();
+      // suffix counts: warp w < 8 owns bins [32w, 32w+32)
+      uint32_t suf = 0;
+      if (warp < 8) {
+        suf = hist[warp * 32 + lane];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          uint32_t n = __shfl_down_sync(0xffffffffu, suf, off);
+          if (lane + off < 32) suf += n;
+        }
+        if (lane == 0) bin_tot[warp] = suf;  // all bins of this warp
       }
-      if (threadIdx.x < 256) {
-        const uint32_t b = threadIdx.x;
-        if (suffix[b] >= (uint32_t)k && suffix[b + 1] < (uint32_t)k) sel_bin = b;
+      __syncthreads();
+      if (warp < 8) {
+        uint32_t higher = 0;  // candidates in bins of higher warps
+        for (int w2 = warp + 1; w2 < 8; ++w2) higher += bin_tot[w2];
+        const uint32_t ge = suf + higher;                                   // digit >= bin
+        const uint32_t gt = ge - hist[warp * 32 + lane];                    // digit > bin
+        if (ge >= (uint32_t)k && gt < (uint32_t)k) {
+          sel_bin = warp * 32 + lane;
+          sel_above = gt;
+        }
       }
       __syncthreads();
       const uint32_t b = sel_bin;
-      k -= (int)suffix[b + 1];
+      k -= (int)sel_above;
       prefix |= b << shift;
       pmask |= 255u << shift;
+      for (int bb = threadIdx.x; bb < 257; bb += kSelThreads) hist[bb] = 0;
       __syncthreads();
     }
     tau = prefix;
     need_eq = k;
   }
 
-  // 3. keep flags and compaction in pool (= position) order
-  const int chunk = (L + kSelThreads - 1) / kSelThreads;
-  const int j0 = min(L, threadIdx.x * chunk), j1 = min(L, j0 + chunk);
-  uint32_t gt = 0, eq = 0;
-  if (!keep_all) {
-    for (int j = j0; j < j1; ++j) {
-      const uint32_t u = score_bits(sc[j]);
-      gt += u > tau;
-      eq += u == tau;
-    }
+  // 3. keep flags and compaction in pool (= position) order, 512 candidates
+  //    per round: a block-wide scan gives each kept candidate its slot, so
+  //    consecutive threads write consecutive slots (coalesced stores)
+  __shared__ int base_kept, base_eq;
+  if (threadIdx.x == 0) {
+    base_kept = 0;
+    base_eq = 0;
   }
-  // L <= 65535 (host-checked), so both counts fit 16 bits
-  const uint32_t packed = block_exclusive_scan(gt | (eq << 16), warp_tot);
-  const int gt_before = packed & 0xffffu;
-  int eq_seen = packed >> 16;
-  int dst = keep_all ? j0 : gt_before + min(eq_seen, need_eq);
-  for (int j = j0; j < j1; ++j) {
-    bool keep = keep_all;
-    if (!keep_all) {
-      const uint32_t u = score_bits(sc[j]);
-      if (u > tau) keep = true;
-      else if (u == tau) keep = eq_seen++ < need_eq;
+  __syncthreads();
+  for (int j0 = 0; j0 < L; j0 += kSelThreads) {
+    const int j = j0 + threadIdx.x;
+    // kept and tied candidates before this round (read before the scan's barriers)
+    const int bk = base_kept, be = base_eq;
+    uint32_t is_gt = 0, is_eq = 0;
+    if (j < L) {
+      if (keep_all) {
+        is_gt = 1;
+      } else {
+        const uint32_t u = score_bits(sc[j]);
+        is_gt = u > tau;
+        is_eq = u == tau;
+      }
     }
-    if (!keep || dst >= a.B) continue;
-    for (int g = G0; g < G1; ++g) {
-      const long long row = ((long long)s * a.Hkv + g) * a.B;
-      const int p = j < a.m ? a.pos_c[row + j] : a.pos_f[(long long)s * a.T + (j - a.m)];
-      a.idx[row + dst] = j;
-      a.pos_new[row + dst] = p;
-      a.score_new[row + dst] = sc[j];
+    const uint32_t packed = block_exclusive_scan(is_gt | (is_eq << 16), warp_tot);
+    const int eq_rank = be + (int)(packed >> 16);  // tied candidates before j
+    const bool keep = is_gt || (is_eq && eq_rank < need_eq);
+    const int dst = bk + (int)(packed & 0xffffu) + (min(eq_rank, need_eq) - min(be, need_eq));
+    if (keep && dst < a.B) a.idx[((long long)s * a.Hkv + G0) * a.B + dst] = j;
+    // the last thread of the round holds the round's totals
+    if (threadIdx.x == kSelThreads - 1) {
+      const int gt_all = (int)(packed & 0xffffu) + (int)is_gt;
+      const int eq_all = (int)(packed >> 16) + (int)is_eq;
+      base_kept = bk + gt_all + (min(be + eq_all, need_eq) - min(be, need_eq));
+      base_eq = be + eq_all;
     }
-    ++dst;
+    __syncthreads();
   }
 }
 
-// Copies 16-byte vectors.  Work item = (stream, KV head, output row, vector);
-// rows [0, m_new) gather C_n, rows [m_new, m_new + T) append the frame to D.
-__global__ void __launch_bounds__(256) gather_append_kernel(GatherArgs a) {
-  const int vec_per_row = a.row_bytes / 16;
-  const int rows = a.m_new + a.T;
-  const long long total = (long long)a.S * a.Hkv * rows * vec_per_row;
-  for (long long w = blockIdx.x * (long long)blockDim.x + threadIdx.x; w < total;
-       w += (long long)gridDim.x * blockDim.x) {
-    const int vec = (int)(w % vec_per_row);
-    long long r = w / vec_per_row;
-    const int row = (int)(r % rows);
-    r /= rows;
-    const int g = (int)(r % a.Hkv);
-    const int s = (int)(r / a.Hkv);
-    const long long sg = (long long)s * a.Hkv + g;
-    const char* ksrc;
-    const char* vsrc;
-    char* kdst;
-    char* vdst;
-    if (row < a.m_new) {
-      const int j = a.idx[sg * a.B + row];
-      if (j < 0 || j >= a.m + a.T) continue;  // never taken for a well-formed kept list
-      if (j < a.m) {
-        const long long off = (sg * a.B + j) * a.row_bytes;
-        ksrc = static_cast<const char*>(a.kc) + off;
-        vsrc = static_cast<const char*>(a.vc) + off;
-      } else {
-        const long long off = (((long long)s * a.T + (j - a.m)) * a.Hkv + g) * a.row_bytes;
-        ksrc = static_cast<const char*>(a.kf) + off;
-        vsrc = static_cast<const char*>(a.vf) + off;
-      }
-      const long long doff = (sg * a.B + row) * a.row_bytes;
-      kdst = static_cast<char*>(a.kc_new) + doff;
-      vdst = static_cast<char*>(a.vc_new) + doff;
-    } else {
-      const int t = row - a.m_new;
-      const long long off = (((long long)s * a.T + t) * a.Hkv + g) * a.row_bytes;
-      ksrc = static_cast<const char*>(a.kf) + off;
-      vsrc = static_cast<const char*>(a.vf) + off;
-      const long long doff = (sg * a.max_tok + a.d_len + t) * a.row_bytes;
-      kdst = static_cast<char*>(a.kd) + doff;
-      vdst = static_cast<char*>(a.vd) + doff;
-      if (g == 0 && vec == 0) a.pos_d[(long long)s * a.max_tok + a.d_len + t] = a.pos_f[(long long)s * a.T + t];
+// One 16-byte vector per thread and step of the grid-stride loop, two steps
+// unrolled so that two kept-index loads and then two row loads are in flight
+// before any store.  Output row r of (stream, KV head): r < m_new gathers C_n
+// from the pool, r >= m_new appends frame token r - m_new to D.  A row pair (K
+// and V) is 2 * row_bytes / 16 vectors.
+__device__ __forceinline__ bool gather_vec(const GatherArgs& a, int v, int per_row, int vpr, int rows,
+                                           const int4** src, int4** dst) {
+  const int rr = v / per_row;
+  int e = v - rr * per_row;
+  const bool isv = e >= vpr;
+  if (isv) e -= vpr;
+  const int row = rr % rows;
+  const int sg = rr / rows;  // s * Hkv + g
+  const int g = sg % a.Hkv;
+  const int s = sg / a.Hkv;
+  const char* sbase;
+  char* dbase;
+  if (row < a.m_new) {
+    const int gsel = a.global ? 0 : g;
+    const int j = __ldg(a.idx + ((long long)s * a.Hkv + gsel) * a.B + row);
+    if (j < 0 || j >= a.m + a.T) return false;  // never taken for a well-formed kept list
+    if (!isv && e == 0) {  // the row's position and score, once per (stream, KV head, slot)
+      a.pos_new[(long long)sg * a.B + row] =
+          j < a.m ? __ldg(a.pos_c + (long long)sg * a.B + j) : __ldg(a.pos_f + (long long)s * a.T + (j - a.m));
+      a.score_new[(long long)sg * a.B + row] = __ldg(a.pool_score + ((long long)s * a.Hkv + gsel) * a.pool_g + j);
     }
-    const int4 kv = __ldg(reinterpret_cast<const int4*>(ksrc) + vec);
-    const int4 vv = __ldg(reinterpret_cast<const int4*>(vsrc) + vec);
-    reinterpret_cast<int4*>(kdst)[vec] = kv;
-    reinterpret_cast<int4*>(vdst)[vec] = vv;
+    if (j < a.m) {
+      sbase = static_cast<const char*>(isv ? a.vc : a.kc) + ((long long)sg * a.B + j) * a.row_bytes;
+    } else {
+      sbase = static_cast<const char*>(isv ? a.vf : a.kf) +
+              (((long long)s * a.T + (j - a.m)) * a.Hkv + g) * a.row_bytes;
+    }
+    dbase = static_cast<char*>(isv ? a.vc_new : a.kc_new) + ((long long)sg * a.B + row) * a.row_bytes;
+  } else {
+    const int t = row - a.m_new;
+    sbase = static_cast<const char*>(isv ? a.vf : a.kf) + (((long long)s * a.T + t) * a.Hkv + g) * a.row_bytes;
+    dbase = static_cast<char*>(isv ? a.vd : a.kd) + ((long long)sg * a.max_tok + a.d_len + t) * a.row_bytes;
+    if (g == 0 && !isv && e == 0)
+      a.pos_d[(long long)s * a.max_tok + a.d_len + t] = __ldg(a.pos_f + (long long)s * a.T + t);
+  }
+  *src = reinterpret_cast<const int4*>(sbase) + e;
+  *dst = reinterpret_cast<int4*>(dbase) + e;
+  return true;
+}
+
+__global__ void __launch_bounds__(256) gather_append_kernel(GatherArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  const int vpr = a.row_bytes / 16;
+  const int per_row = 2 * vpr;
+  const int rows = a.m_new + a.T;
+  const int total = a.S * a.Hkv * rows * per_row;
+  const int stride = gridDim.x * blockDim.x;
+  for (int v0 = blockIdx.x * blockDim.x + threadIdx.x; v0 < total; v0 += 2 * stride) {
+    const int v1 = v0 + stride;
+    const int4* s0 = nullptr;
+    const int4* s1 = nullptr;
+    int4* d0 = nullptr;
+    int4* d1 = nullptr;
+    const bool ok0 = gather_vec(a, v0, per_row, vpr, rows, &s0, &d0);
+    const bool ok1 = v1 < total && gather_vec(a, v1, per_row, vpr, rows, &s1, &d1);
+    int4 x0, x1;
+    if (ok0) x0 = __ldg(s0);
+    if (ok1) x1 = __ldg(s1);
+    if (ok0) *d0 = x0;
+    if (ok1) *d1 = x1;
   }
 }
 
 }  // namespace
 
-cudaError_t launch_select(const SelectArgs& a, int S, cudaStream_t st) {
+cudaError_t launch_select(const SelectArgs& a, int S, cudaStream_t st, bool pdl) {
   const int L = a.m + a.T;
   const int n_groups = a.global ? 1 : a.Hkv;
-  const size_t smem = (size_t)L * sizeof(float);
+  const size_t smem = (size_t)L * (sizeof(float) + sizeof(int));
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(select_topb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
   }
-  select_topb_kernel<<<dim3(n_groups, S), kSelThreads, smem, st>>>(a);
-  return cudaGetLastError();
+  return launch_kernel(select_topb_kernel, dim3(n_groups, S), dim3(kSelThreads), smem, st, pdl, a);
 }
 
-cudaError_t launch_gather(const GatherArgs& a, int n_sm, cudaStream_t st) {
-  const long long total = (long long)a.S * a.Hkv * (a.m_new + a.T) * (a.row_bytes / 16);
-  if (total == 0) return cudaSuccess;
-  long long blocks = (total + 255) / 256;
-  const long long cap = (long long)n_sm * 8;
+cudaError_t launch_gather(const GatherArgs& a, int n_sm, cudaStream_t st, bool pdl) {
+  const long long vecs = (long long)a.S * a.Hkv * (a.m_new + a.T) * 2 * (a.row_bytes / 16);
+  if (vecs == 0) return cudaSuccess;
+  long long blocks = (vecs + 2 * 256 - 1) / (2 * 256);  // two vectors per thread
+  const long long cap = (long long)n_sm * 8;           // one resident wave at 8 blocks per SM
   if (blocks > cap) blocks = cap;
-  gather_append_kernel<<<(int)blocks, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  return launch_kernel(gather_append_kernel, dim3((unsigned)blocks), dim3(256), 0, st, pdl, a);
 }
 
 }  // namespace skv

@@ -55,7 +55,7 @@ struct statekv_handle {
   float* pool_score = nullptr;  // [S][Hkv][B+T]
   int32_t* idx = nullptr;       // [S][Hkv][max(B,1)]
   int* dev_err = nullptr;       // kernel error word (bounded-wait timeouts)
-  float* o_part = nullptr;      // attention key-split partials (bf16 path)
+  __nv_bfloat16* o_part = nullptr;  // attention key-split partials (bf16 path)
   float* ml_part = nullptr;
   int max_split = 1;
   // staging for statekv_prefill_frame_host (allocated on first use)
@@ -123,10 +123,13 @@ int check_shape(statekv_t h, int S, int Hq, int Hkv, int d, int T, int B, int ma
   if (select != STATEKV_SELECT_GLOBAL && select != STATEKV_SELECT_PER_KV_HEAD)
     return set_err(h, STATEKV_ERR_INVALID_ARG, "bad select_mode %d", select);
   if (d != 64 && d != 128) return set_err(h, STATEKV_ERR_UNSUPPORTED, "head dim %d not in {64,128}", d);
-  if ((long long)B + T > 49152)
-    return set_err(h, STATEKV_ERR_UNSUPPORTED, "pool B+T=%lld above 49152", (long long)B + T);
+  if ((long long)B + T > 28672)
+    return set_err(h, STATEKV_ERR_UNSUPPORTED, "pool B+T=%lld above 28672", (long long)B + T);
   if ((long long)max_frames * T > (1LL << 30))
     return set_err(h, STATEKV_ERR_UNSUPPORTED, "max_frames*T too large");
+  // bf16 score pass keeps the row statistics of one KV group in shared memory
+  if (dtype == STATEKV_BF16 && (Hq / Hkv) * ((T + 127) / 128) > 112)
+    return set_err(h, STATEKV_ERR_UNSUPPORTED, "bf16 path needs (Hq/Hkv)*ceil(T/128) <= 112");
   return STATEKV_OK;
 }
 
@@ -238,7 +241,7 @@ namespace {
 // demand (one buffer per device, guarded by a mutex).
 std::mutex g_fc_mu;
 struct FcScratch {
-  float* o = nullptr;
+  __nv_bfloat16* o = nullptr;
   float* ml = nullptr;
   int* err = nullptr;
   size_t o_bytes = 0, ml_bytes = 0;
@@ -273,7 +276,7 @@ int full_causal_tc(const void* q, const void* k, const void* v, int n_seq, int N
   {
     std::lock_guard<std::mutex> lk(g_fc_mu);
     FcScratch& sc = g_fc[dev];
-    const size_t ob = ta.n_split > 1 ? (size_t)n_seq * Hq * ta.n_split * N * d * 4 : 16;
+    const size_t ob = ta.n_split > 1 ? (size_t)n_seq * Hq * ta.n_split * N * d * 2 : 16;
     const size_t mb = ta.n_split > 1 ? (size_t)n_seq * Hq * ta.n_split * N * 4 : 16;
     if (!sc.err && cudaMalloc((void**)&sc.err, 16) == cudaSuccess) cudaMemset(sc.err, 0, 16);
     if (sc.o_bytes < ob) {
@@ -363,7 +366,7 @@ int statekv_create_batched(statekv_t* out, int n_streams, int Hq, int Hkv, int d
   if (dtype == STATEKV_BF16) {
     h->max_split = skv::attn_tc_splits(n_streams, Hq, Hkv, T, B, h->n_sm);
     if (h->max_split > 1 &&
-        ((rc = dev_alloc(h, (void**)&h->o_part, (size_t)n_streams * Hq * h->max_split * T * d * 4)) ||
+        ((rc = dev_alloc(h, (void**)&h->o_part, (size_t)n_streams * Hq * h->max_split * T * d * 2)) ||
          (rc = dev_alloc(h, (void**)&h->ml_part, (size_t)n_streams * Hq * h->max_split * T * 4)))) {
       g_free_error = h->err;
       statekv_destroy(h);
@@ -461,13 +464,13 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
     ta.err = h->dev_err;
     {
       StageScope sc(h, st, STATEKV_STAGE_ATTENTION);
-      if ((e = skv::launch_attn_tc(tq, tkc, tvc, tkf, tvf, ta, d, st)) != cudaSuccess)
+      if ((e = skv::launch_attn_tc(tq, tkc, tvc, tkf, tvf, ta, d, st, true)) != cudaSuccess)
         return launch_err(h, e, "attention");
       sc.done();
     }
     if (ta.n_split > 1) {
       StageScope sc(h, st, STATEKV_STAGE_ATTENTION_COMBINE);
-      if ((e = skv::launch_attn_combine(ta, d, st)) != cudaSuccess) return launch_err(h, e, "attention combine");
+      if ((e = skv::launch_attn_combine(ta, d, st, true)) != cudaSuccess) return launch_err(h, e, "attention combine");
       sc.done();
     }
   } else {
@@ -517,7 +520,7 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
     ta.scale_log2 = scale_log2;
     ta.err = h->dev_err;
     StageScope sc(h, st, STATEKV_STAGE_SCORE);
-    if ((e = skv::launch_score_tc(tq, tkc, tkf, ta, d, st)) != cudaSuccess) return launch_err(h, e, "score");
+    if ((e = skv::launch_score_tc(tq, tkc, tkf, ta, d, st, true)) != cudaSuccess) return launch_err(h, e, "score");
     sc.done();
   } else {
     StageScope sc(h, st, STATEKV_STAGE_SCORE);
@@ -534,8 +537,6 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
   se.pos_c = L->posc[cur];
   se.pos_f = pos;
   se.idx = h->idx;
-  se.pos_new = L->posc[nxt];
-  se.score_new = L->scorec[nxt];
   se.Hkv = Hkv;
   se.m = m;
   se.T = T;
@@ -543,7 +544,7 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
   se.global = h->select == STATEKV_SELECT_GLOBAL;
   {
     StageScope sc(h, st, STATEKV_STAGE_SELECT);
-    if ((e = skv::launch_select(se, S, st)) != cudaSuccess) return launch_err(h, e, "select");
+    if ((e = skv::launch_select(se, S, st, true)) != cudaSuccess) return launch_err(h, e, "select");
     sc.done();
   }
 
@@ -560,6 +561,11 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
   ga.vd = L->vd;
   ga.pos_d = L->posd;
   ga.pos_f = pos;
+  ga.pos_c = se.pos_c;
+  ga.pool_score = se.pool_score;
+  ga.pos_new = L->posc[nxt];
+  ga.score_new = L->scorec[nxt];
+  ga.pool_g = se.part_g;
   ga.Hkv = Hkv;
   ga.T = T;
   ga.B = B;
@@ -572,7 +578,7 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
   ga.S = S;
   {
     StageScope sc(h, st, STATEKV_STAGE_GATHER);
-    if ((e = skv::launch_gather(ga, h->n_sm, st)) != cudaSuccess) return launch_err(h, e, "gather");
+    if ((e = skv::launch_gather(ga, h->n_sm, st, true)) != cudaSuccess) return launch_err(h, e, "gather");
     sc.done();
   }
 

@@ -77,7 +77,7 @@ extern "C" int statekv_step_noalloc(int Hq, int Hkv, int d, int T, int B, int dt
   const size_t part_b = round256((size_t)Hkv * pool * 4);
   const size_t idx_b = round256((size_t)Hkv * (B > 0 ? B : 1) * 4);
   const size_t need = lse_b + 2 * part_b + idx_b;
-  if (need > kNoAllocScratchBytes || pool > 49152)
+  if (need > kNoAllocScratchBytes || pool > 28672)
     return fail(STATEKV_ERR_UNSUPPORTED,
                 "shape needs %zu bytes of step scratch; statekv_step_noalloc has %zu (use statekv_create)",
                 need, kNoAllocScratchBytes);
@@ -168,8 +168,6 @@ extern "C" int statekv_step_noalloc(int Hq, int Hkv, int d, int T, int B, int dt
   se.pos_c = posc;
   se.pos_f = pos;
   se.idx = idx;
-  se.pos_new = posc_new;
-  se.score_new = scorec_new;
   se.Hkv = Hkv;
   se.m = m;
   se.T = T;
@@ -190,6 +188,11 @@ extern "C" int statekv_step_noalloc(int Hq, int Hkv, int d, int T, int B, int dt
   ga.vd = vd;
   ga.pos_d = posd;
   ga.pos_f = pos;
+  ga.pos_c = se.pos_c;
+  ga.pool_score = se.pool_score;
+  ga.pos_new = posc_new;
+  ga.score_new = scorec_new;
+  ga.pool_g = se.part_g;
   ga.Hkv = Hkv;
   ga.T = T;
   ga.B = B;
