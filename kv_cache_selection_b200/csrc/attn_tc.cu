@@ -24,10 +24,12 @@
 // partials that attn_combine merges, or out and lse directly when unsplit.
 //
 // Warp roles (384 threads): warp 0 TMA producer, warp 1 TMEM allocator + MMA
-// issuer, warps 4..7 softmax of tile A, warps 8..11 softmax of tile B.
+// issuer, warps 4..7 softmax of tile A, warps 8..11 softmax of tile B (warp w
+// reads TMEM lanes 32*(w%4) .. +31, so each group covers all 128 rows).
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_common.cuh"
+#include "merge.cuh"
 
 
 namespace skv {
@@ -36,6 +38,12 @@ using namespace tc;
 
 constexpr int kSlots = 4;        // K/V ring slots (each one 128-key tile)
 constexpr int kThreads = 384;
+// registers: launched at 168 per thread (384 x 168 = 64512); warpgroup 0
+// (producer, MMA issuer, two idle warps) drops to 72 and the two softmax
+// warpgroups rise to 216: 128 x 72 + 256 x 216 = 64512.
+constexpr int kRegsLow = 72;
+constexpr int kRegsHigh = 216;
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * 168, "register split exceeds the launch");
 constexpr float kRescaleLog2 = 8.0f;
 
 template <int D>
@@ -142,6 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto col_s = [](int x) { return (uint32_t)(x * 128); };
   auto col_o = [](int x) { return (uint32_t)(256 + x * 128); };
 
+  if (warp < 4) regs_dec<kRegsLow>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -238,6 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax
+    regs_inc<kRegsHigh>();
     const int x = (warp - 4) >> 2;  // 0: tile A, 1: tile B
     const TileInfo ti = x == 0 ? tA : tB;
     const int nX = x == 0 ? nA : nB;
@@ -259,21 +269,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       int lim = is_c ? a.m - base : (a.causal ? min(a.T, i + 1) : a.T) - base;
       lim = max(0, min(128, lim));
       const bool masked = __any_sync(0xffffffffu, lim < 128);
-      // pass 1: row max of the scaled logits
-      float mx = -INFINITY;
+      // the whole 128-column row of S in one batch of TMEM loads
+      uint32_t sv[128];
+      tmem_ld32(t_s + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+      tmem_ld32(t_s + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
+      tmem_ld32(t_s + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+      tmem_ld_wait();
+      if (masked) {
 #pragma unroll
-      for (int c0 = 0; c0 < 4; ++c0) {
-        uint32_t v[32];
-        tmem_ld32(t_s + c0 * 32, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
-          float sv = __uint_as_float(v[jj]) * c;
-          if (masked && c0 * 32 + jj >= lim) sv = -INFINITY;
-          mx = fmaxf(mx, sv);
-        }
+        for (int jj = 0; jj < 128; ++jj)
+          if (jj >= lim) sv[jj] = __float_as_uint(-INFINITY);
       }
-      float m_new = fmaxf(m_used, mx);
+      // row max of the raw logits (c > 0), three inputs per instruction
+      float mx = __uint_as_float(sv[0]);
+#pragma unroll
+      for (int jj = 1; jj < 127; jj += 2) mx = max3f(mx, __uint_as_float(sv[jj]), __uint_as_float(sv[jj + 1]));
+      mx = fmaxf(mx, __uint_as_float(sv[127]));
+      float m_new = fmaxf(m_used, mx * c);
       if (m_new == -INFINITY) m_new = 0.f;  // nothing visible yet in this row
       if (j == 0) {
         m_used = m_new;
@@ -296,22 +309,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (need) m_used = m_new;
         }
       }
-      // pass 2: P = exp2(S*c - m_used) as bf16 into the first 64 columns
+      // P = exp2(S*c - m_used) (masked entries hold -inf -> 0), as bf16 into
+      // the first 64 columns of the same TMEM region
       float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
       for (int c0 = 0; c0 < 4; ++c0) {
-        uint32_t v[32];
-        tmem_ld32(t_s + c0 * 32, v);
-        tmem_ld_wait();
         uint32_t pk[16];
 #pragma unroll
         for (int jj = 0; jj < 16; ++jj) {
-          float p0 = ex2_approx(fmaf(__uint_as_float(v[2 * jj]), c, -m_used));
-          float p1 = ex2_approx(fmaf(__uint_as_float(v[2 * jj + 1]), c, -m_used));
-          if (masked) {
-            if (c0 * 32 + 2 * jj >= lim) p0 = 0.f;
-            if (c0 * 32 + 2 * jj + 1 >= lim) p1 = 0.f;
-          }
+          const float p0 = ex2_approx(fmaf(__uint_as_float(sv[c0 * 32 + 2 * jj]), c, -m_used));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(sv[c0 * 32 + 2 * jj + 1]), c, -m_used));
           ls0 += p0;
           ls1 += p1;
           pk[jj] = pack_bf16x2(p0, p1);
@@ -385,60 +392,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Merge of key-split partials.  One thread per (query row, 8-element chunk of
-// d): it reads the row's n_split log2-sum-exps and its chunk of every split's
-// O/l at once (independent loads), weights them by 2^(ml_u - max) and writes
-// the bf16 result; chunk 0 also writes the row's natural-log lse.
-constexpr int kMaxSplit = 8;
-
 template <int D>
-__global__ void __launch_bounds__(256) attn_combine_kernel(AttnTcArgs a) {
+__global__ void __launch_bounds__(256) attn_combine_kernel(MergeArgs a) {
   pdl_wait();
   pdl_trigger();
-  constexpr int kChunks = D / 8;
-  const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  const int rows = a.S * a.Hq * a.T;
-  if (t >= rows * kChunks) return;
-  const int chunk = t % kChunks;
-  const int rw = t / kChunks;
-  const int i = rw % a.T;
-  const int sh = rw / a.T;  // s * Hq + h
-  const int h = sh % a.Hq, s = sh / a.Hq;
-  const long long prow0 = (long long)sh * a.n_split * a.T + i;
-  float ml[kMaxSplit];
-  uint4 raw[kMaxSplit];
-#pragma unroll
-  for (int u = 0; u < kMaxSplit; ++u) {
-    if (u < a.n_split) {
-      ml[u] = __ldg(a.ml_part + prow0 + (long long)u * a.T);
-      raw[u] = __ldg(reinterpret_cast<const uint4*>(a.o_part + (prow0 + (long long)u * a.T) * D) + chunk);
-    }
-  }
-  float mx = -INFINITY;
-#pragma unroll
-  for (int u = 0; u < kMaxSplit; ++u)
-    if (u < a.n_split) mx = fmaxf(mx, ml[u]);
-  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  float wsum = 0.f;
-#pragma unroll
-  for (int u = 0; u < kMaxSplit; ++u) {
-    if (u < a.n_split) {
-      const float w = ml[u] == -INFINITY ? 0.f : ex2_approx(ml[u] - mx);
-      wsum += w;
-      const __nv_bfloat16* v = reinterpret_cast<const __nv_bfloat16*>(&raw[u]);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] += w * __bfloat162float(v[e]);
-    }
-  }
-  const float inv = 1.f / wsum;
-  uint4 o;
-  uint32_t* op = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-  for (int e = 0; e < 4; ++e) op[e] = pack_bf16x2(acc[2 * e] * inv, acc[2 * e + 1] * inv);
-  __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + s * a.out_s + (long long)i * a.out_row +
-                        (long long)h * D;
-  reinterpret_cast<uint4*>(orow)[chunk] = o;
-  if (chunk == 0 && a.lse) a.lse[s * a.lse_s + (long long)h * a.T + i] = (mx + __log2f(wsum)) * kLn2;
+  merge_chunk<D>(a, blockIdx.x * blockDim.x + threadIdx.x);
 }
 
 }  // namespace
@@ -452,7 +410,7 @@ int attn_tc_splits(int S, int Hq, int Hkv, int T, int m, int n_sm) {
   int split = n_sm / units;
   if (split < 1) split = 1;
   if (split > nk) split = nk;
-  if (split > kMaxSplit) split = kMaxSplit;
+  if (split > kMaxSplit) split = kMaxSplit;  // the merge holds at most kMaxSplit partials
   return split;
 }
 
@@ -477,11 +435,29 @@ cudaError_t launch_attn_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kc, co
   return cudaGetLastError();
 }
 
+MergeArgs merge_args(const AttnTcArgs& a, int d) {
+  MergeArgs m{};
+  m.out = a.out;
+  m.out_s = a.out_s;
+  m.out_row = a.out_row;
+  m.lse = a.lse;
+  m.lse_s = a.lse_s;
+  m.o_part = a.o_part;
+  m.ml_part = a.ml_part;
+  m.S = a.S;
+  m.Hq = a.Hq;
+  m.T = a.T;
+  m.n_split = a.n_split;
+  m.d = d;
+  return m;
+}
+
 cudaError_t launch_attn_combine(const AttnTcArgs& a, int d, cudaStream_t st, bool pdl) {
+  const MergeArgs m = merge_args(a, d);
   const long long rows = (long long)a.S * a.Hq * a.T;
   const int blocks = (int)((rows * (d / 8) + 255) / 256);
-  if (d == 128) return launch_kernel(attn_combine_kernel<128>, dim3(blocks), dim3(256), 0, st, pdl, a);
-  return launch_kernel(attn_combine_kernel<64>, dim3(blocks), dim3(256), 0, st, pdl, a);
+  if (d == 128) return launch_kernel(attn_combine_kernel<128>, dim3(blocks), dim3(256), 0, st, pdl, m);
+  return launch_kernel(attn_combine_kernel<64>, dim3(blocks), dim3(256), 0, st, pdl, m);
 }
 
 }  // namespace skv

@@ -77,7 +77,21 @@ struct ScoreArgs {
   float scale_log2;
 };
 
-// Top-B selection over the pool of one (stream, selection group).
+// Merge of the attention's key-split partials into out and lse.
+struct MergeArgs {
+  void* out;                     // out[s][i][h][dd] bf16
+  long long out_s;
+  int out_row;
+  float* lse;                    // [S][Hq][T] natural log, may be null
+  long long lse_s;
+  const __nv_bfloat16* o_part;   // [S][Hq][n_split][T][d] O/l per split
+  const float* ml_part;          // [S][Hq][n_split][T] log2-sum-exp
+  int S, Hq, T, n_split, d;
+};
+
+// Top-B selection over the pool of one (stream, selection group).  The same
+// launch carries extra blocks that append the frame to the detailed state and
+// merge the attention's key-split partials (neither is on the path to C_n).
 struct SelectArgs {
   const float* part;      // part[s][g][j], j < m + T
   long long part_s;
@@ -87,6 +101,18 @@ struct SelectArgs {
   const int32_t* pos_f;   // frame positions [s][T]
   int32_t* idx;           // out [s][g][B] kept pool indices, ascending (row 0 in global mode)
   int Hkv, m, T, B, global;
+  int n_sel_blocks;       // blocks [0, n_sel_blocks): one per (stream, selection group)
+  // D append: frame [s][t][g][d] -> D [s][g][max_tok][d] at token d_len
+  int n_app_blocks;
+  const void* kf;
+  const void* vf;
+  void* kd;
+  void* vd;
+  int32_t* pos_d;         // [s][max_tok]
+  int row_bytes, d_len, max_tok, S;
+  // key-split merge (n_mrg_blocks > 0 only for the bf16 attention with splits)
+  int n_mrg_blocks;
+  MergeArgs mrg;
 };
 
 // Gather of the kept rows into the next C buffer plus the append of the

@@ -43,8 +43,10 @@ int encode_tmap_bf16_4d(CUtensorMap* map, const void* base, const uint64_t dims[
 // Tensor-core score pass (bf16): the three maps cover q [S][T][Hq][d],
 // K_C [S][Hkv][B][d] and the frame keys [S][T][Hkv][d], boxes of 64 x 128 rows.
 struct ScoreTcArgs {
-  const float* lse;  // [S][Hq][T] natural log
+  const float* lse;  // [S][Hq][T] natural log (read when n_split == 1)
   long long lse_s;
+  const float* ml_part;  // [S][Hq][n_split][T] log2-sum-exp per key split (n_split > 1)
+  int n_split;
   float* part;       // [S][Hkv][pool]
   long long part_s;
   int part_g;
@@ -74,6 +76,7 @@ cudaError_t launch_attn_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kc, co
                            const CUtensorMap& tm_kf, const CUtensorMap& tm_vf, const AttnTcArgs& a, int d,
                            cudaStream_t st, bool pdl = false);
 cudaError_t launch_attn_combine(const AttnTcArgs& a, int d, cudaStream_t st, bool pdl = false);
+MergeArgs merge_args(const AttnTcArgs& a, int d);
 
 // Message for statekv_last_error(NULL) (errors of calls without a handle).
 void set_free_error(const char* msg);

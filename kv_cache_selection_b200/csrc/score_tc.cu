@@ -14,8 +14,10 @@
 // Each epilogue thread owns one key's TMEM lane, so the column sum of P is a
 // private running sum: no shuffles, no atomics, deterministic.
 //
-// Warp roles (320 threads): warp 0 TMA producer, warp 1 TMEM allocator + MMA
-// issuer, warps 2..9 epilogue (two warpgroups split each chunk's columns).
+// Warp roles (384 threads): warp 0 TMA producer, warp 1 TMEM allocator + MMA
+// issuer, warps 4..11 epilogue: two warpgroups (each covers the 128 TMEM
+// lanes) take alternate chunks, so two chunks are in the epilogue while the
+// MMA fills the next two of the four TMEM accumulators.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_common.cuh"
@@ -25,8 +27,18 @@ namespace {
 using namespace tc;
 
 constexpr int kStages = 4;
-constexpr int kEpiWarps = 8;
-constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kGroups = 4;                      // epilogue warpgroups (take chunks round robin)
+constexpr int kEpiWarps = 4 * kGroups;
+constexpr int kThreads = 128 + 32 * kEpiWarps;  // warpgroup 0: producer, MMA, two idle warps
+// exponentials of columns with (col & 15) >= kPolyFrom run on the FMA pipe
+// (polynomial), the rest on MUFU; 16 = all on MUFU
+constexpr int kPolyFrom = 16;
+// registers: the launch gives each thread kRegsLaunch; warpgroup 0 drops to
+// kRegsLow and the epilogue warpgroups rise to kRegsHigh within that total
+constexpr int kRegsLaunch = (65536 / kThreads) / 8 * 8 > 168 ? 168 : (65536 / kThreads) / 8 * 8;
+constexpr int kRegsLow = kGroups == 2 ? 72 : 56;
+constexpr int kRegsHigh = ((kThreads * kRegsLaunch - 128 * kRegsLow) / (128 * kGroups)) / 8 * 8;
+static_assert(128 * kRegsLow + 128 * kGroups * kRegsHigh <= kThreads * kRegsLaunch, "register split exceeds the launch");
 
 template <int D>
 struct Smem {
@@ -35,10 +47,10 @@ struct Smem {
   static constexpr int kTileBytes = kAtoms * kAtomBytes;
   static constexpr int kK = 0;
   static constexpr int kQ = kK + kTileBytes;
-  static constexpr int kRed = kQ + kStages * kTileBytes;  // 128 floats
-  static constexpr int kBar = kRed + 128 * 4;
-  // k_full, q_full[kStages], q_empty[kStages], acc_full[2], acc_empty[2], done
-  static constexpr int kNumBars = 1 + 2 * kStages + 4 + 1;
+  static constexpr int kRed = kQ + kStages * kTileBytes;  // (kGroups - 1) x 128 floats
+  static constexpr int kBar = kRed + (kGroups - 1) * 128 * 4;
+  // k_full, q_full[kStages], q_empty[kStages], acc_full[4], acc_empty[4], done
+  static constexpr int kNumBars = 1 + 2 * kStages + 8 + 1;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kLse = (kAbort + 4 + 15) & ~15;    // [G][n_ic*128] row statistics follow
@@ -69,8 +81,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar_qfull = [&](int st) { return sb + L::kBar + 8u * (1 + st); };
   auto bar_qempty = [&](int st) { return sb + L::kBar + 8u * (1 + kStages + st); };
   auto bar_accfull = [&](int b) { return sb + L::kBar + 8u * (1 + 2 * kStages + b); };
-  auto bar_accempty = [&](int b) { return sb + L::kBar + 8u * (3 + 2 * kStages + b); };
-  const uint32_t bar_done = sb + L::kBar + 8u * (5 + 2 * kStages);
+  auto bar_accempty = [&](int b) { return sb + L::kBar + 8u * (5 + 2 * kStages + b); };
+  const uint32_t bar_done = sb + L::kBar + 8u * (9 + 2 * kStages);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
 
@@ -80,16 +92,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_qfull(st), 1);
       mbar_init(bar_qempty(st), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < 4; ++b) {
       mbar_init(bar_accfull(b), 1);
-      mbar_init(bar_accempty(b), kEpiWarps);
+      mbar_init(bar_accempty(b), 4);  // the four warps of the group that owns chunk c's buffer
     }
     mbar_init(bar_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), 256);  // two 128-column f32 accumulators
+    tmem_alloc(smem_u32(tmem_slot), 512);  // four 128-column f32 accumulators
     tmem_relinquish();
   }
   fence_before_sync();
@@ -99,6 +111,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_wait();
   pdl_trigger();
 
+  if (warp < 4) regs_dec<kRegsLow>();
   if (warp == 0) {
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
@@ -131,9 +144,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc = idesc_bf16(128, 128, false, false);
       bool ok = mbar_wait(bar_k, 0, a.err, kErrWaitLoad, abort_flag);
       for (int c = 0; ok && c < n_chunks; ++c) {
-        const int st = c % kStages, buf = c & 1;
+        const int st = c % kStages, buf = c & 3;
         if (!mbar_wait(bar_qfull(st), (c / kStages) & 1, a.err, kErrWaitLoad, abort_flag)) break;
-        if (!mbar_wait(bar_accempty(buf), ((c >> 1) & 1) ^ 1, a.err, kErrWaitAccFree, abort_flag)) break;
+        if (!mbar_wait(bar_accempty(buf), ((c >> 2) & 1) ^ 1, a.err, kErrWaitAccFree, abort_flag)) break;
         fence_after_sync();
         const uint32_t qbase = sb + L::kQ + st * L::kTileBytes;
 #pragma unroll
@@ -149,77 +162,120 @@ __global__ void __launch_bounds__(kThreads, 1)
       drain_wait(bar_done, 0, a.err);
     }
     __syncwarp();
-  } else {
-    const int ew = warp - 2;              // 0..7
+  } else if (warp >= 4) {
+    regs_inc<kRegsHigh>();
+    const int ew = warp - 4;              // 0..7
     const int quarter = warp & 3;         // TMEM lane quarter this warp may access
-    const int half = ew >> 2;             // which 64 columns of each chunk
+    const int half = ew >> 2;             // group: takes chunks half, half + kGroups, ...
     const int row = quarter * 32 + lane;  // key row within the tile
     const int key = r0 + row;
-    // row statistics of the whole group in log2 units, +inf past the frame
+    // row statistics of the whole group in log2 units, negated, -inf past the
+    // frame: log2-sum-exp = max + log2(sum 2^(ml_u - max)) over the
+    // attention's key splits (or the stored lse when unsplit).  Loads of a
+    // thread's rows are issued before any is used.
     const int tpad = n_ic * 128;
     float* lse_all = reinterpret_cast<float*>(smem + L::kLse);
-    for (int e = threadIdx.x - 64; e < G * tpad; e += 32 * kEpiWarps) {
-      const int hh = e / tpad, i = e % tpad;
-      lse_all[e] = i < a.T ? a.lse[s * a.lse_s + (long long)(g * G + hh) * a.T + i] * kLog2e : INFINITY;
+    constexpr int kRowsPerThread = 4;
+    for (int e0 = threadIdx.x - 128; e0 < G * tpad; e0 += 32 * kEpiWarps * kRowsPerThread) {
+      float vals[kRowsPerThread][8];
+#pragma unroll
+      for (int q = 0; q < kRowsPerThread; ++q) {
+        const int e = e0 + q * 32 * kEpiWarps;
+        const int hh = e / tpad, i = e % tpad;
+        const bool valid = e < G * tpad && i < a.T;
+        const long long rowbase = (long long)(s * a.Hq + g * G + hh);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          vals[q][u] = -INFINITY;
+          if (valid && a.n_split > 1 && u < a.n_split) vals[q][u] = a.ml_part[(rowbase * a.n_split + u) * a.T + i];
+        }
+        if (valid && a.n_split <= 1) vals[q][0] = a.lse[rowbase * a.T + i] * kLog2e;
+      }
+#pragma unroll
+      for (int q = 0; q < kRowsPerThread; ++q) {
+        const int e = e0 + q * 32 * kEpiWarps;
+        if (e >= G * tpad) continue;
+        float mx = vals[q][0];
+#pragma unroll
+        for (int u = 1; u < 8; ++u) mx = fmaxf(mx, vals[q][u]);
+        float l2 = mx;
+        if (a.n_split > 1 && mx > -INFINITY) {
+          float ssum = 0.f;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) ssum += vals[q][u] == -INFINITY ? 0.f : ex2_approx(vals[q][u] - mx);
+          l2 = mx + __log2f(ssum);
+        }
+        // rows past the frame have no statistics: -inf makes their weight 0
+        lse_all[e] = mx == -INFINITY ? -INFINITY : -l2;
+      }
     }
     named_bar_sync(2, 32 * kEpiWarps);
     float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
     bool ok = true;
-    for (int c = 0; c < n_chunks; ++c) {
-      const int buf = c & 1;
+    for (int c = half; c < n_chunks; c += kGroups) {
+      const int buf = c & 3;
       const int hh = c / per_head;
       const int i0 = (ic_min + c % per_head) * 128;
-      const int cbase = i0 + half * 64;
-      const float* lse2 = lse_all + hh * tpad + cbase;
+      const float* lse2 = lse_all + hh * tpad + i0;
       uint32_t got = 1;
-      if (lane == 0) got = mbar_wait(bar_accfull(buf), (c >> 1) & 1, a.err, kErrWaitAcc, abort_flag) ? 1u : 0u;
+      if (lane == 0) got = mbar_wait(bar_accfull(buf), (c >> 2) & 1, a.err, kErrWaitAcc, abort_flag) ? 1u : 0u;
       got = __shfl_sync(0xffffffffu, got, 0);
       if (!got) {
         ok = false;
         break;
       }
       fence_after_sync();
-      // some of this warp's columns precede some key of the tile (warp-uniform)
-      const bool diag = !is_c && a.causal && (cbase < r0 + 127);
-      uint32_t rr[2][32];
-      tmem_ld32(tmem_addr(tmem, quarter * 32, buf * 128 + half * 64), rr[0]);
-      tmem_ld32(tmem_addr(tmem, quarter * 32, buf * 128 + half * 64 + 32), rr[1]);
-      tmem_ld_wait();
+      // some columns of this chunk precede some key of the tile (frame-causal),
+      // or lie past the frame
+      const bool diag = !is_c && a.causal && (i0 < r0 + 127);
+      const bool need_mask = diag || i0 + 128 > a.T;
+#pragma unroll 1
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t rr[2][32];
+        tmem_ld32(tmem_addr(tmem, quarter * 32, buf * 128 + hf * 64), rr[0]);
+        tmem_ld32(tmem_addr(tmem, quarter * 32, buf * 128 + hf * 64 + 32), rr[1]);
+        tmem_ld_wait();
 #pragma unroll
-      for (int q32 = 0; q32 < 2; ++q32) {
-        const uint32_t* r = rr[q32];
-        const float4* l4 = reinterpret_cast<const float4*>(lse2 + q32 * 32);
+        for (int qq = 0; qq < 2; ++qq) {
+          const int q = hf * 2 + qq;
+          const float4* l4 = reinterpret_cast<const float4*>(lse2 + q * 32);
 #pragma unroll
-        for (int j4 = 0; j4 < 8; ++j4) {
-          const float4 lv = l4[j4];
-          float p0 = ex2_approx(fmaf(__uint_as_float(r[4 * j4 + 0]), a.scale_log2, -lv.x));
-          float p1 = ex2_approx(fmaf(__uint_as_float(r[4 * j4 + 1]), a.scale_log2, -lv.y));
-          float p2 = ex2_approx(fmaf(__uint_as_float(r[4 * j4 + 2]), a.scale_log2, -lv.z));
-          float p3 = ex2_approx(fmaf(__uint_as_float(r[4 * j4 + 3]), a.scale_log2, -lv.w));
-          if (diag) {
-            const int i = cbase + q32 * 32 + 4 * j4;  // frame token `key` is seen by rows i >= key
-            p0 = key <= i + 0 ? p0 : 0.f;
-            p1 = key <= i + 1 ? p1 : 0.f;
-            p2 = key <= i + 2 ? p2 : 0.f;
-            p3 = key <= i + 3 ? p3 : 0.f;
+          for (int j4 = 0; j4 < 8; ++j4) {
+            const float4 lv = l4[j4];  // -lse2 of 4 columns
+            const float x0 = fmaf(__uint_as_float(rr[qq][4 * j4 + 0]), a.scale_log2, lv.x);
+            float p0 = (((4 * j4 + 0) & 15) >= kPolyFrom) ? exp2_poly<4>(x0) : ex2_approx(x0);
+            const float x1 = fmaf(__uint_as_float(rr[qq][4 * j4 + 1]), a.scale_log2, lv.y);
+            float p1 = (((4 * j4 + 1) & 15) >= kPolyFrom) ? exp2_poly<4>(x1) : ex2_approx(x1);
+            const float x2 = fmaf(__uint_as_float(rr[qq][4 * j4 + 2]), a.scale_log2, lv.z);
+            float p2 = (((4 * j4 + 2) & 15) >= kPolyFrom) ? exp2_poly<4>(x2) : ex2_approx(x2);
+            const float x3 = fmaf(__uint_as_float(rr[qq][4 * j4 + 3]), a.scale_log2, lv.w);
+            float p3 = (((4 * j4 + 3) & 15) >= kPolyFrom) ? exp2_poly<4>(x3) : ex2_approx(x3);
+            if (need_mask) {
+              // frame token `key` is seen by rows i >= key (frame-causal); rows past T do not exist
+              const int i = i0 + q * 32 + 4 * j4;
+              p0 = (i + 0 < a.T && (!diag || key <= i + 0)) ? p0 : 0.f;
+              p1 = (i + 1 < a.T && (!diag || key <= i + 1)) ? p1 : 0.f;
+              p2 = (i + 2 < a.T && (!diag || key <= i + 2)) ? p2 : 0.f;
+              p3 = (i + 3 < a.T && (!diag || key <= i + 3)) ? p3 : 0.f;
+            }
+            acc0 += p0;
+            acc1 += p1;
+            acc2 += p2;
+            acc3 += p3;
           }
-          acc0 += p0;
-          acc1 += p1;
-          acc2 += p2;
-          acc3 += p3;
         }
       }
       fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_accempty(buf));
     }
-    // combine the two column halves of each key row
+    // combine the groups' partial sums of each key row (fixed order)
     float tot = (acc0 + acc1) + (acc2 + acc3);
     float* red = reinterpret_cast<float*>(smem + L::kRed);
-    if (half == 1) red[row] = tot;
+    if (half > 0) red[(half - 1) * 128 + row] = tot;
     named_bar_sync(1, 32 * kEpiWarps);
     if (half == 0 && ok && !*abort_flag) {
-      tot += red[row];
+      for (int gr = 1; gr < kGroups; ++gr) tot += red[(gr - 1) * 128 + row];
       const bool valid = is_c ? key < a.m : key < a.T;
       if (valid) {
         const int j = is_c ? key : a.m + key;
@@ -231,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     fence_after_sync();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 

@@ -12,6 +12,7 @@
 // C_{n-1} is, and every frame position exceeds all earlier ones).
 #include "common.cuh"
 #include "kernels.h"
+#include "merge.cuh"
 
 namespace skv {
 namespace {
@@ -56,19 +57,51 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* w
 // pool's scores (L floats).  Radix select on 8-bit digits, most significant
 // first; each pass is a histogram (warp-aggregated shared atomics) and a
 // suffix count over the 256 bins done with warp shuffles.
+// Appends frame token vectors to D: one 16-byte vector per thread.
+__device__ __forceinline__ void append_vec(const SelectArgs& a, int v) {
+  const int vpr = a.row_bytes / 16;
+  const int per_row = 2 * vpr;  // K and V
+  const int rr = v / per_row;   // (s, t, g) row of the frame
+  if (rr >= a.S * a.T * a.Hkv) return;
+  int e = v - rr * per_row;
+  const bool isv = e >= vpr;
+  if (isv) e -= vpr;
+  const int g = rr % a.Hkv;
+  const int st = rr / a.Hkv;  // s * T + t
+  const int t = st % a.T, s = st / a.T;
+  const long long src = (long long)rr * a.row_bytes;
+  const long long dst = (((long long)s * a.Hkv + g) * a.max_tok + a.d_len + t) * a.row_bytes;
+  const int4 x = __ldg(reinterpret_cast<const int4*>(static_cast<const char*>(isv ? a.vf : a.kf) + src) + e);
+  reinterpret_cast<int4*>(static_cast<char*>(isv ? a.vd : a.kd) + dst)[e] = x;
+  if (g == 0 && !isv && e == 0) a.pos_d[(long long)s * a.max_tok + a.d_len + t] = __ldg(a.pos_f + st);
+}
+
 __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) {
   extern __shared__ float sc[];
   __shared__ uint32_t hist[257];
   __shared__ uint32_t bin_tot[8];
   __shared__ uint32_t warp_tot[32];
   __shared__ uint32_t sel_bin, sel_above;
-  const int grp = blockIdx.x, s = blockIdx.y;
+  pdl_wait();
+  pdl_trigger();
+  if ((int)blockIdx.x >= a.n_sel_blocks) {
+    // extra blocks: D append, then the merge of key-split partials
+    const int b = blockIdx.x - a.n_sel_blocks;
+    if (b < a.n_app_blocks) {
+      append_vec(a, b * kSelThreads + threadIdx.x);
+    } else {
+      const int t = (b - a.n_app_blocks) * kSelThreads + threadIdx.x;
+      if (a.mrg.d == 128) merge_chunk<128>(a.mrg, t);
+      else merge_chunk<64>(a.mrg, t);
+    }
+    return;
+  }
+  const int n_groups = a.global ? 1 : a.Hkv;
+  const int grp = blockIdx.x % n_groups, s = blockIdx.x / n_groups;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int L = a.m + a.T;
   const int G0 = a.global ? 0 : grp;
   const int G1 = a.global ? a.Hkv : grp + 1;
-  pdl_wait();
-  pdl_trigger();
 
   // 1. scores of the pool (global mode sums the KV groups in a fixed order)
   //    and the pool positions, staged in shared memory; every load of a
@@ -233,11 +266,7 @@ __device__ __forceinline__ bool gather_vec(const GatherArgs& a, int v, int per_r
     }
     dbase = static_cast<char*>(isv ? a.vc_new : a.kc_new) + ((long long)sg * a.B + row) * a.row_bytes;
   } else {
-    const int t = row - a.m_new;
-    sbase = static_cast<const char*>(isv ? a.vf : a.kf) + (((long long)s * a.T + t) * a.Hkv + g) * a.row_bytes;
-    dbase = static_cast<char*>(isv ? a.vd : a.kd) + ((long long)sg * a.max_tok + a.d_len + t) * a.row_bytes;
-    if (g == 0 && !isv && e == 0)
-      a.pos_d[(long long)s * a.max_tok + a.d_len + t] = __ldg(a.pos_f + (long long)s * a.T + t);
+    return false;  // rows past m_new do not exist
   }
   *src = reinterpret_cast<const int4*>(sbase) + e;
   *dst = reinterpret_cast<int4*>(dbase) + e;
@@ -249,7 +278,7 @@ __global__ void __launch_bounds__(256) gather_append_kernel(GatherArgs a) {
   pdl_trigger();
   const int vpr = a.row_bytes / 16;
   const int per_row = 2 * vpr;
-  const int rows = a.m_new + a.T;
+  const int rows = a.m_new;
   const int total = a.S * a.Hkv * rows * per_row;
   const int stride = gridDim.x * blockDim.x;
   for (int v0 = blockIdx.x * blockDim.x + threadIdx.x; v0 < total; v0 += 2 * stride) {
@@ -270,20 +299,32 @@ __global__ void __launch_bounds__(256) gather_append_kernel(GatherArgs a) {
 
 }  // namespace
 
-cudaError_t launch_select(const SelectArgs& a, int S, cudaStream_t st, bool pdl) {
+cudaError_t launch_select(const SelectArgs& a_in, int S, cudaStream_t st, bool pdl) {
+  SelectArgs a = a_in;
   const int L = a.m + a.T;
   const int n_groups = a.global ? 1 : a.Hkv;
+  a.n_sel_blocks = n_groups * S;
+  const long long app_vecs = (long long)S * a.T * a.Hkv * 2 * (a.row_bytes / 16);
+  a.n_app_blocks = (int)((app_vecs + kSelThreads - 1) / kSelThreads);
+  a.S = S;
+  if (a.mrg.n_split > 1) {
+    const long long mrg_threads = (long long)a.mrg.S * a.mrg.Hq * a.mrg.T * (a.mrg.d / 8);
+    a.n_mrg_blocks = (int)((mrg_threads + kSelThreads - 1) / kSelThreads);
+  } else {
+    a.n_mrg_blocks = 0;
+  }
   const size_t smem = (size_t)L * (sizeof(float) + sizeof(int));
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(select_topb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
   }
-  return launch_kernel(select_topb_kernel, dim3(n_groups, S), dim3(kSelThreads), smem, st, pdl, a);
+  return launch_kernel(select_topb_kernel, dim3(a.n_sel_blocks + a.n_app_blocks + a.n_mrg_blocks),
+                       dim3(kSelThreads), smem, st, pdl, a);
 }
 
 cudaError_t launch_gather(const GatherArgs& a, int n_sm, cudaStream_t st, bool pdl) {
-  const long long vecs = (long long)a.S * a.Hkv * (a.m_new + a.T) * 2 * (a.row_bytes / 16);
+  const long long vecs = (long long)a.S * a.Hkv * a.m_new * 2 * (a.row_bytes / 16);
   if (vecs == 0) return cudaSuccess;
   long long blocks = (vecs + 2 * 256 - 1) / (2 * 256);  // two vectors per thread
   const long long cap = (long long)n_sm * 8;           // one resident wave at 8 blocks per SM

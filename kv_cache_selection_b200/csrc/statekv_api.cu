@@ -19,7 +19,7 @@
 #include <string>
 #include <vector>
 
-#include "../../include/statekv.h"
+#include "statekv.h"
 #include "kernels.h"
 
 namespace {
@@ -439,6 +439,8 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
   aa.causal = h->mask == STATEKV_MASK_FRAME_CAUSAL;
   aa.scale_log2 = scale_log2;
   CUtensorMap tq, tkc, tkf, tvc, tvf;
+  skv::MergeArgs mrg{};  // key-split merge, run by the select launch (bf16 with splits)
+  int n_split = 1;
   if (h->dtype == STATEKV_BF16) {
     if ((rc = encode_step_maps(h, q, L->kc[cur], k, &tq, &tkc, &tkf, L->vc[cur], v, &tvc, &tvf))) return rc;
     skv::AttnTcArgs ta{};
@@ -468,11 +470,8 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
         return launch_err(h, e, "attention");
       sc.done();
     }
-    if (ta.n_split > 1) {
-      StageScope sc(h, st, STATEKV_STAGE_ATTENTION_COMBINE);
-      if ((e = skv::launch_attn_combine(ta, d, st, true)) != cudaSuccess) return launch_err(h, e, "attention combine");
-      sc.done();
-    }
+    n_split = ta.n_split;
+    if (n_split > 1) mrg = skv::merge_args(ta, d);
   } else {
     StageScope sc(h, st, STATEKV_STAGE_ATTENTION);
     if ((e = skv::launch_attn_simt(aa, h->dtype, d, S, st)) != cudaSuccess) return launch_err(h, e, "attention");
@@ -506,6 +505,8 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
     skv::ScoreTcArgs ta{};
     ta.lse = h->lse;
     ta.lse_s = aa.lse_s;
+    ta.ml_part = h->ml_part;
+    ta.n_split = n_split;
     ta.part = h->part;
     ta.part_s = sa.part_s;
     ta.part_g = pool;
@@ -542,6 +543,15 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
   se.T = T;
   se.B = B;
   se.global = h->select == STATEKV_SELECT_GLOBAL;
+  se.kf = k;
+  se.vf = v;
+  se.kd = L->kd;
+  se.vd = L->vd;
+  se.pos_d = L->posd;
+  se.row_bytes = (int)(d * h->esize);
+  se.d_len = L->frames * T;
+  se.max_tok = h->max_frames * T;
+  se.mrg = mrg;
   {
     StageScope sc(h, st, STATEKV_STAGE_SELECT);
     if ((e = skv::launch_select(se, S, st, true)) != cudaSuccess) return launch_err(h, e, "select");

@@ -63,18 +63,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait for the completion of the phase with the given parity.
+// Bounded wait for the completion of the phase with the given parity.  The
+// abort flag and the clock are checked every 64 polls only, so a waiting
+// thread takes few issue slots from the warps that share its scheduler.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err, int code,
                                           volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
-  while (true) {
+  for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      atomicCAS(err, 0, code);
-      *abort_flag = 1;
-      return false;
+    if ((it & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        atomicCAS(err, 0, code);
+        *abort_flag = 1;
+        return false;
+      }
     }
   }
 }
@@ -206,6 +210,24 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool 
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// Per-warpgroup register reallocation (all 128 threads of a warpgroup execute
+// it).  Increases draw on what other warpgroups released, so the shares must
+// add up to the launch's threads x registers.
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -215,8 +237,8 @@ __device__ __forceinline__ float ex2_approx(float x) {
 // Bounded wait used on teardown paths only: ignores the abort flag.
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, int* err) {
   const unsigned long long t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+  for (uint32_t it = 1; !mbar_try_wait(bar, parity); ++it) {
+    if ((it & 63u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
       atomicCAS(err, 0, kErrWaitDrain);
       return;
     }
@@ -229,6 +251,33 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int* er
   uint32_t ok = 1;
   if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, err, code, abort_flag) ? 1u : 0u;
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// 2^x on the FMA pipe instead of the MUFU unit (for kernels whose
+// exponentials outnumber what MUFU can issue).  Range reduction: j = round(x)
+// by adding 1.5 * 2^23 (the integer lands in the low mantissa bits),
+// f = x - j in [-1/2, 1/2]; 2^f by a polynomial whose coefficients were fitted
+// for minimal relative error on that interval (degree 3: 1.0e-4, degree 4:
+// 2.9e-6, evaluated in float32 Horner form); 2^j is applied by adding j to the
+// exponent field.  x is clamped at -120, so inputs below that give about
+// 2^-120, not 0: callers mask explicitly where exact zeros matter.
+template <int DEG>
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -120.f);
+  const float t = x + 12582912.f;
+  const float j = t - 12582912.f;
+  const float f = x - j;
+  float p;
+  if (DEG == 3) {
+    p = fmaf(f, 0.055008821189403534f, 0.2422107756137848f);
+    p = fmaf(f, p, 0.6932829022407532f);
+  } else {
+    p = fmaf(f, 0.009582837112247944f, 0.05590641498565674f);
+    p = fmaf(f, p, 0.24024099111557007f);
+    p = fmaf(f, p, 0.6931241750717163f);
+  }
+  p = fmaf(f, p, 1.f);
+  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
