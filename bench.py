@@ -149,6 +149,31 @@ def ncu_traffic(kernel_stage, workload):
         return None
 
 
+def dist_max(x: float, device) -> float:
+    """Max of a per-rank number over all ranks (identity without a process group)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return float(x)
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_sum(x: float, device) -> float:
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return float(x)
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+def replica_throughput(local_frames: int, local_ms: float, device) -> tuple:
+    """Whole-job frames/s of independent replicas: all frames over the slowest
+    rank's time.  Returns (value, max_ms)."""
+    max_ms = dist_max(local_ms, device)
+    frames = dist_sum(local_frames, device)
+    return frames / (max_ms / 1e3), max_ms
+
+
 # ------------------------------------------------------------------ our arm --
 def make_frames(wl, n_distinct, stream, dev):
     fr = Syn.gen_frames(wl, n_distinct, stream=stream)
@@ -213,11 +238,7 @@ def run_ours(args, wl):
     stages = h.profile_read()
     h.profile(False)
     ms_steps = [a.elapsed_time(b) for a, b in ev]
-    ms_total = sum(ms_steps)
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_total = float(t.item())
+    value, ms_total = replica_throughput(K, sum(ms_steps), dev)
 
     # ---- end to end through the host-buffer C-ABI call (pinned host memory)
     e2e = None
@@ -261,15 +282,11 @@ def run_ours(args, wl):
             he.prefill_frame_host(0, qh, kh, vh, ph, oh)
             ev2[j][1].record()
         torch.cuda.synchronize()
-        e2e_ms = sum(a.elapsed_time(b) for a, b in ev2)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_value, e2e_ms = replica_throughput(K, sum(a.elapsed_time(b) for a, b in ev2), dev)
         esize = 2 if wl.dtype == "bf16" else 4
         h2d = (wl.T * wl.Hq * wl.d + 2 * wl.T * wl.Hkv * wl.d) * esize + wl.T * 4
         d2h = wl.T * wl.Hq * wl.d * esize
-        e2e = {"value": world * K / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        e2e = {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K,
                "path": "statekv_prefill_frame_host (pinned host buffers, copies on the step's stream)"}
         he.close()
@@ -318,7 +335,7 @@ def run_ours(args, wl):
     h.close()
 
     line = {
-        "metric": METRIC, "value": round(world * K / (ms_total / 1e3), 2), "unit": UNIT,
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT,
         "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": round(ms_total / K, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
         "data": "synthetic",
@@ -372,6 +389,160 @@ def cpu_baseline(wl, h, fr_cpu, n_next, n_distinct, budget_s=20.0, kv_heads=None
             "sample": f"{frames_done} steady-state frames of {wl.name} on {kvh} of {wl.Hkv} KV heads "
                       f"({kvh * G} query heads), float64 numpy oracle, {el:.1f} s; value scaled by "
                       f"{wl.Hkv}/{kvh}"}
+
+
+# ------------------------------------------------------------ report modes --
+def _flush_l2(buf, j):
+    if buf is not None:
+        buf.fill_(j)
+
+
+def _per_frame_times(step_fn, n_frames, flush, dev):
+    """Device time of each step (CUDA events, L2 flushed between steps)."""
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_frames)]
+    torch.cuda.synchronize()
+    for n in range(n_frames):
+        _flush_l2(flush, n)
+        ev[n][0].record()
+        step_fn(n)
+        ev[n][1].record()
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) * 1e3 for a, b in ev]  # us
+
+
+def _flatness(us, first):
+    import numpy as np
+    y = np.asarray(us[first:])
+    x = np.arange(first, len(us))
+    slope = float(np.polyfit(x, y, 1)[0]) if len(y) > 2 else 0.0
+    p50 = float(np.percentile(y, 50))
+    p99 = float(np.percentile(y, 99))
+    return {"from_frame": first, "mean_us": round(float(y.mean()), 2), "p50_us": round(p50, 2),
+            "p99_us": round(p99, 2), "p99_over_p50": round(p99 / p50, 3),
+            "slope_us_per_frame": round(slope, 5),
+            "slope_over_512_frames_pct": round(100 * slope * 512 / p50, 2)}
+
+
+def run_flatness(args):
+    """8B-class layer over all 512 frames: per-frame latency vs frame index."""
+    from kv_cache_selection_b200 import statekv as SKV
+    wl = Syn.workload("8b_layer")
+    dev = torch.device("cuda")
+    q, k, v, pos = Syn.gen_frames_device(wl, wl.frames, device=dev)
+    h = SKV.StateKV(wl.Hq, wl.Hkv, wl.d, wl.T, wl.B, max_frames=wl.frames + 8, dtype=wl.dtype)
+    h.reserve_layers(1)
+    out = torch.empty_like(q[0])
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.int32, device=dev)
+    us = _per_frame_times(lambda n: h.prefill_frame(0, q[n], k[n], v[n], pos[n], out), wl.frames, flush, dev)
+    fill = math.ceil(wl.B / wl.T)
+    rep = {"report": "flatness", "workload": "8b_layer (512 frames, B=4096), device-drawn synthetic frames",
+           "l2": "flushed between frames", "fill_frames": fill,
+           "fill_us": [round(x, 1) for x in us[:fill]], "steady": _flatness(us, fill),
+           "per_frame_us_every_32": [round(x, 1) for x in us[::32]]}
+    h.close()
+    print(json.dumps(rep), flush=True)
+
+
+def run_stack(args):
+    """28 independent 8B-class layers, layers in order per frame, 128 frames."""
+    from kv_cache_selection_b200 import statekv as SKV
+    wl = Syn.workload("8b_stack")
+    dev = torch.device("cuda")
+    n_frames = args.stack_frames or wl.frames
+    layers = [Syn.gen_frames_device(wl, n_frames, layer=l, device=dev) for l in range(wl.layers)]
+    h = SKV.StateKV(wl.Hq, wl.Hkv, wl.d, wl.T, wl.B, max_frames=n_frames, dtype=wl.dtype)
+    h.reserve_layers(wl.layers)
+    out = torch.empty_like(layers[0][0][0])
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.int32, device=dev)
+
+    def frame(n):
+        for l, (q, k, v, pos) in enumerate(layers):
+            h.prefill_frame(l, q[n], k[n], v[n], pos[n], out)
+
+    us = _per_frame_times(frame, n_frames, flush, dev)
+    fill = math.ceil(wl.B / wl.T)
+    d_bytes = wl.layers * n_frames * wl.T * wl.Hkv * wl.d * 2 * 2
+    rep = {"report": "stack", "workload": f"8b_stack: {wl.layers} layers x {n_frames} frames, B={wl.B}",
+           "per_frame_us_all_layers": _flatness(us, fill),
+           "per_frame_layer_us": round(_flatness(us, fill)["p50_us"] / wl.layers, 2),
+           "frames_per_s_per_layer": round(1e6 / (_flatness(us, fill)["p50_us"] / wl.layers), 1),
+           "detailed_state_bytes_K_plus_V": d_bytes,
+           "per_frame_us_every_8": [round(x, 1) for x in us[::8]]}
+    h.close()
+    print(json.dumps(rep), flush=True)
+
+
+def run_sweep(args):
+    """8B layer shape, 4 streams per launch: cumulative StateKV prefill cost
+    against full_causal_prefill over the same N*256 tokens."""
+    from kv_cache_selection_b200 import statekv as SKV
+    wl = Syn.workload("8b_sweep")
+    dev = torch.device("cuda")
+    S = wl.streams
+    n_max = max(args.sweep_frames)
+    per = [Syn.gen_frames_device(wl, n_max, stream=s, device=dev) for s in range(S)]
+    # [S][n][T][H][d] so that the first N frames of a stream are one sequence
+    Q = torch.stack([p[0] for p in per])
+    Kt = torch.stack([p[1] for p in per])
+    V = torch.stack([p[2] for p in per])
+    P = torch.stack([p[3] for p in per])
+    del per
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.int32, device=dev)
+    res = {"report": "sweep", "workload": f"8b layer shape, {S} streams per launch, frames {args.sweep_frames}",
+           "statekv": {}, "full_causal_us": {}, "crossover_frames": {}, "analytic_crossover_frames_3_passes": {}}
+    fc = {}
+    for N in args.sweep_frames:
+        ntok = N * wl.T
+        q = Q[:, :N].reshape(S, ntok, wl.Hq, wl.d).contiguous()
+        kk = Kt[:, :N].reshape(S, ntok, wl.Hkv, wl.d).contiguous()
+        vv = V[:, :N].reshape(S, ntok, wl.Hkv, wl.d).contiguous()
+        out = torch.empty_like(q)
+        SKV.full_causal_prefill(q, kk, vv, out=out, with_lse=False)  # warm-up
+        torch.cuda.synchronize()
+        _flush_l2(flush, N)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        SKV.full_causal_prefill(q, kk, vv, out=out, with_lse=False)
+        e1.record()
+        torch.cuda.synchronize()
+        fc[N] = e0.elapsed_time(e1) * 1e3
+        res["full_causal_us"][N] = round(fc[N], 1)
+        del out, q, kk, vv
+    for B in args.sweep_b:
+        h = SKV.StateKV(wl.Hq, wl.Hkv, wl.d, wl.T, B, max_frames=n_max, dtype=wl.dtype, n_streams=S)
+        h.reserve_layers(1)
+        qs = torch.empty((S, wl.T, wl.Hq, wl.d), dtype=wl.torch_dtype, device=dev)
+        ks = torch.empty((S, wl.T, wl.Hkv, wl.d), dtype=wl.torch_dtype, device=dev)
+        vs = torch.empty_like(ks)
+        ps = torch.empty((S, wl.T), dtype=torch.int32, device=dev)
+        out = torch.empty_like(qs)
+        times = []
+        for n in range(n_max):
+            qs.copy_(Q[:, n]); ks.copy_(Kt[:, n]); vs.copy_(V[:, n]); ps.copy_(P[:, n])
+            _flush_l2(flush, n)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            h.prefill_frame(0, qs, ks, vs, ps, out)
+            e1.record()
+            times.append((e0, e1))
+        torch.cuda.synchronize()
+        us = [a.elapsed_time(b) * 1e3 for a, b in times]
+        cum, acc = {}, 0.0
+        for n, t in enumerate(us):
+            acc += t
+            if n + 1 in args.sweep_frames:
+                cum[n + 1] = round(acc, 1)
+        fill = math.ceil(B / wl.T)
+        res["statekv"][B] = {"cumulative_us": cum, "steady_step_us_4_streams": _flatness(us, fill)["p50_us"]}
+        cross = None
+        for N in sorted(args.sweep_frames):
+            if cum[N] <= fc[N]:
+                cross = N
+                break
+        res["crossover_frames"][B] = cross
+        res["analytic_crossover_frames_3_passes"][B] = round(3 * (B + wl.T / 2) / wl.T, 1)
+        h.close()
+    print(json.dumps(res), flush=True)
 
 
 # ------------------------------------------------------------ reference arm --
@@ -440,10 +611,18 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle time")
+    ap.add_argument("--mode", choices=["headline", "flatness", "stack", "sweep"], default="headline",
+                    help="headline: the contract's JSON line; others: report lines")
+    ap.add_argument("--stack-frames", type=int, default=0)
+    ap.add_argument("--sweep-frames", type=int, nargs="+", default=[32, 64, 128, 256, 512, 1024])
+    ap.add_argument("--sweep-b", type=int, nargs="+", default=[1024, 2048, 4096])
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     wl = Syn.workload(args.workload)
+    if args.mode != "headline":
+        {"flatness": run_flatness, "stack": run_stack, "sweep": run_sweep}[args.mode](args)
+        return
     if args.impl == "reference":
         run_reference(args, wl)
     else:

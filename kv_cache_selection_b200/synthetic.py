@@ -185,3 +185,44 @@ def gen_tokens(wl: Workload, n_tokens: int, layer: int = 0, stream: int = 0):
     k = torch.cat([f[1] for f in fr])[:n_tokens].contiguous()
     v = torch.cat([f[2] for f in fr])[:n_tokens].contiguous()
     return q, k, v
+
+
+def gen_frames_device(wl: Workload, n_frames: int, layer: int = 0, stream: int = 0,
+                      device="cuda", start: int = 0):
+    """The same recipe drawn with torch's device generator, for timing runs that
+    need many frames (values differ from gen_frame's; parity checks use
+    gen_frame).  Returns stacked q [n][T][Hq][d], k/v [n][T][Hkv][d] and
+    pos [n][T] on `device`."""
+    T, Hq, Hkv, d = wl.T, wl.Hq, wl.Hkv, wl.d
+    g = torch.Generator(device=device)
+    g.manual_seed(wl.layer_seed(layer) * 1_000_003 + stream * 10_007 + start)
+    q = torch.randn((n_frames, T, Hq, d), generator=g, device=device, dtype=torch.float32)
+    k = torch.randn((n_frames, T, Hkv, d), generator=g, device=device, dtype=torch.float32)
+    v = torch.randn((n_frames, T, Hkv, d), generator=g, device=device, dtype=torch.float32)
+    pos = (torch.arange(start * T, (start + n_frames) * T, device=device, dtype=torch.int64)
+           .view(n_frames, T))
+    if wl.dist == "sinks":
+        s = 1.0 / float(np.sqrt(d))
+        q *= s
+        k *= s
+        v *= s
+    half = d // 2
+    inv_freq = 10000.0 ** (-torch.arange(half, device=device, dtype=torch.float64) * 2.0 / d)
+    ang = pos.to(torch.float64)[..., None] * inv_freq          # [n][T][half]
+    cos = torch.cos(ang).to(torch.float32)[:, :, None, :]
+    sin = torch.sin(ang).to(torch.float32)[:, :, None, :]
+
+    def rope(x):
+        x1, x2 = x[..., :half], x[..., half:]
+        return torch.cat([x1 * cos - x2 * sin, x2 * cos + x1 * sin], dim=-1)
+
+    q = rope(q)
+    k = rope(k)
+    if wl.dist == "sinks" and wl.n_sinks:
+        u = torch.from_numpy(sink_direction(wl, layer)).to(device=device, dtype=torch.float32)
+        q += 1.5 * u
+        idx = torch.stack([torch.randperm(T, generator=g, device=device)[: wl.n_sinks] for _ in range(n_frames)])
+        rows = torch.arange(n_frames, device=device)[:, None].expand_as(idx)
+        k[rows, idx] += 4.0 * u
+    dt = wl.torch_dtype
+    return q.to(dt), k.to(dt), v.to(dt), pos.to(torch.int32)

@@ -1,0 +1,72 @@
+"""The multi-GPU bench path (independent replicas, one per rank) on CPU with
+the gloo backend: the whole-job value is all ranks' frames over the slowest
+rank's device time, and every rank sees the same numbers.  Also: the
+reference arm does no work on ranks other than 0."""
+
+import os
+import socket
+import sys
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, results):
+    sys.path.insert(0, ROOT)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    torch.distributed.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import bench
+        # rank r processed 100*(r+1) frames in 10*(r+1) ms of device time
+        value, max_ms = bench.replica_throughput(100 * (rank + 1), 10.0 * (rank + 1), "cpu")
+        results[rank] = (value, max_ms)
+    finally:
+        torch.distributed.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2])
+def test_replica_throughput_gloo(world):
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        results = mgr.dict()
+        procs = [ctx.Process(target=_worker, args=(r, world, port, results)) for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(timeout=120)
+            assert p.exitcode == 0
+        got = dict(results)
+    frames = sum(100 * (r + 1) for r in range(world))
+    slowest = 10.0 * world
+    for r in range(world):
+        value, max_ms = got[r]
+        assert max_ms == pytest.approx(slowest)
+        assert value == pytest.approx(frames / (slowest / 1e3))
+
+
+def test_single_process_is_identity():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert not torch.distributed.is_initialized()
+    value, max_ms = bench.replica_throughput(50, 25.0, "cpu")
+    assert max_ms == 25.0 and value == pytest.approx(2000.0)
+
+
+def test_reference_arm_other_ranks_exit_without_work(monkeypatch, capsys):
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    bench.main(["--impl", "reference", "--steps", "3", "--warmup", "3"])
+    assert capsys.readouterr().out == ""

@@ -240,3 +240,51 @@ def test_full_causal_prefill_large_sampled_rows():
     ref_out, ref_lse = O.causal_attention_rows(q, k, v, rows)
     P.check_out(out[rows], ref_out, "bf16")
     P.check_lse(lse[:, rows], ref_lse, "bf16")
+
+
+@cuda
+def test_8b_stack_layers_interleaved():
+    """28 independent 8B-class layers processed in order per frame (the
+    full-stack workload): per-step parity on sampled (layer, frame) pairs across
+    the fill phase and eviction; every layer's D holds its own frames."""
+    S = _skv()
+    wl = Syn.workload("8b_stack")
+    n_frames = 18
+    checks = {(0, 0), (13, 16), (27, 17), (5, 17)}
+    dev = torch.device("cuda")
+    h = S.StateKV(wl.Hq, wl.Hkv, wl.d, wl.T, wl.B, max_frames=n_frames, dtype="bf16")
+    h.reserve_layers(wl.layers)
+    for n in range(n_frames):
+        for layer in range(wl.layers):
+            q, k, v, pos = Syn.gen_frame(wl, n, layer=layer)
+            check = (layer, n) in checks
+            C_before = _clone_C(h.get_compressed(layer)) if (check and n > 0) else None
+            out = h.prefill_frame(layer, q.to(dev), k.to(dev), v.to(dev), pos.to(dev))
+            if not check:
+                continue
+            torch.cuda.synchronize()
+            st = P.oracle_state_from_gpu(C_before) if C_before is not None else O.LayerState.empty(wl.Hkv, wl.d)
+            _, res = O.statekv_step(st, q, k, v, pos.numpy(), wl.B)
+            P.check_out(out, res["out"], "bf16", what=f"layer {layer} frame {n}")
+            stats = h.step_stats()
+            P.check_lse(stats["lse"][0], res["lse"], "bf16")
+            P.check_scores(stats["pool_score"][0, :1, :stats["pool_len"]], res["score"][:1], wl.Hq * wl.T)
+            C = h.get_compressed(layer)
+            P.check_selection(C["pos"][0, 0, :C["len"]].cpu().numpy(), res["kept"][0], res["score"][0],
+                              res["pool_pos"][0], wl.B)
+    for layer in (0, 27):
+        D = h.get_detailed(layer)
+        assert D["len"] == n_frames * wl.T
+        k_last = Syn.gen_frame(wl, n_frames - 1, layer=layer)[1]
+        assert torch.equal(D["k"][0, :, (n_frames - 1) * wl.T:n_frames * wl.T].cpu(), k_last.transpose(0, 1))
+    assert h.device_status() == 0
+    h.close()
+
+
+@cuda
+def test_8b_sweep_shape_four_streams():
+    """The sweep workload's launch shape: 4 streams per call at the 8B layer
+    shape, with B=1024 so eviction starts at frame 4."""
+    wl = Syn.workload("8b_sweep", B=1024, frames=6)
+    r = run_stream_parity(wl, wl.frames, check={0, 4, 5}, n_streams=4)
+    assert r["checked"] == 3 * 4  # three frames, four streams
