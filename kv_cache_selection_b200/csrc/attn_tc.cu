@@ -122,6 +122,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
 
   if (threadIdx.x == 0) {
+    // the maps are kernel parameters, not outputs of the preceding kernel
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_kc);
+    tma_prefetch_desc(&tm_vc);
+    tma_prefetch_desc(&tm_kf);
+    tma_prefetch_desc(&tm_vf);
     mbar_init(bar_q, 1);
     for (int sl = 0; sl < kSlots; ++sl) {
       mbar_init(bar_kvfull(sl), 1);
@@ -154,7 +160,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
       const int nq = (nA > 0 ? 1 : 0) + (nB > 0 ? 1 : 0);
       if (nq) {
         mbar_arrive_expect_tx(bar_q, nq * L::kTileBytes);
@@ -191,26 +196,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);
       constexpr uint32_t id_o = idesc_bf16(128, D, false, true);
       const int nX[2] = {nA, nB};
-      auto slot_addr = [&](int idx) { return sb + L::kKV + (idx % kSlots) * L::kTileBytes; };
+      // Descriptors are formed once; per MMA only the start address (bits
+      // 0..13, 16-byte units) advances, which never carries into the other
+      // fields.
+      const uint64_t dq0 = sdesc_sw128(sb + L::kQ, 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(sb + L::kKV, 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(sb + L::kKV, L::kAtomBytes, 1024);
+      auto slot16 = [&](int idx) { return (uint64_t)((idx % kSlots) * (L::kTileBytes >> 4)); };
       auto wait_slot = [&](int idx) {
         return mbar_wait(bar_kvfull(idx % kSlots), (idx / kSlots) & 1, a.err, kErrWaitLoad, abort_flag);
       };
       auto issue_s = [&](int x, int j) {  // S_x = Q_x K_j^T
-        const uint32_t qb = sb + L::kQ + x * L::kTileBytes, kbase = slot_addr(2 * j);
+        const uint64_t dq = dq0 + (uint64_t)((x * L::kTileBytes) >> 4), dk = dk0 + slot16(2 * j);
+        const uint32_t d_tmem = tmem + col_s(x);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::kAtomBytes + (kk & 3) * 32;
-          mma_ss(tmem + col_s(x), sdesc_sw128(qb + off, 16, 1024), sdesc_sw128(kbase + off, 16, 1024), id_s,
-                 kk > 0 ? 1u : 0u);
+          const uint64_t off = (uint64_t)(((kk >> 2) * L::kAtomBytes + (kk & 3) * 32) >> 4);
+          mma_ss(d_tmem, dq + off, dk + off, id_s, kk > 0 ? 1u : 0u);
         }
         mma_commit(bar_sfull(x));
       };
       auto issue_pv = [&](int x, int j) {  // O_x += P_x V_j
-        const uint32_t vbase = slot_addr(2 * j + 1);
+        const uint64_t dv = dv0 + slot16(2 * j + 1);
+        const uint32_t d_tmem = tmem + col_o(x), a_tmem = tmem + col_s(x);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + col_o(x), tmem + col_s(x) + kk * 8, sdesc_sw128(vbase + kk * 2048, L::kAtomBytes, 1024),
-                 id_o, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(d_tmem, a_tmem + kk * 8, dv + (uint64_t)((kk * 2048) >> 4), id_o, (j > 0 || kk > 0) ? 1u : 0u);
         if (j == nX[x] - 1) mma_commit(bar_odone(x));
       };
       bool ok = mbar_wait(bar_q, 0, a.err, kErrWaitLoad, abort_flag) && wait_slot(0);
@@ -260,7 +271,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_used = -INFINITY, l = 0.f;
     bool ok = ti.valid;
     for (int j = 0; ok && j < nX; ++j) {
-      if (!(ok = warp_wait(bar_sfull(x), j & 1, a.err, kErrWaitAcc, abort_flag))) break;
+      // S_j is on the critical chain: spin (a suspending wait wakes later)
+      if (!(ok = warp_spin_wait(bar_sfull(x), j & 1, a.err, kErrWaitAcc, abort_flag))) break;
       fence_after_sync();
       const int k = kb + j;
       const bool is_c = k < a.nC;
@@ -281,11 +293,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int jj = 0; jj < 128; ++jj)
           if (jj >= lim) sv[jj] = __float_as_uint(-INFINITY);
       }
-      // row max of the raw logits (c > 0), three inputs per instruction
-      float mx = __uint_as_float(sv[0]);
+      // row max of the raw logits (c > 0): eight independent chains
+      float m8[8];
 #pragma unroll
-      for (int jj = 1; jj < 127; jj += 2) mx = max3f(mx, __uint_as_float(sv[jj]), __uint_as_float(sv[jj + 1]));
-      mx = fmaxf(mx, __uint_as_float(sv[127]));
+      for (int q8 = 0; q8 < 8; ++q8) {
+        m8[q8] = __uint_as_float(sv[16 * q8]);
+#pragma unroll
+        for (int jj = 1; jj < 15; jj += 2)
+          m8[q8] = max3f(m8[q8], __uint_as_float(sv[16 * q8 + jj]), __uint_as_float(sv[16 * q8 + jj + 1]));
+        m8[q8] = fmaxf(m8[q8], __uint_as_float(sv[16 * q8 + 15]));
+      }
+      const float mx = fmaxf(fmaxf(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5])), fmaxf(m8[6], m8[7]));
       float m_new = fmaxf(m_used, mx * c);
       if (m_new == -INFINITY) m_new = 0.f;  // nothing visible yet in this row
       if (j == 0) {

@@ -245,6 +245,45 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, int* e
   }
 }
 
+// Non-blocking probe of a phase (never suspends the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait in which every lane of the warp spins on test_wait: it sees a
+// completed phase sooner than a suspending try_wait, at the cost of issue
+// slots, so it suits warps on the critical path.  The result is warp-uniform.
+__device__ __forceinline__ bool warp_spin_wait(uint32_t bar, uint32_t parity, int* err, int code,
+                                               volatile int* abort_flag) {
+  unsigned long long t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    if (__any_sync(0xffffffffu, mbar_test_wait(bar, parity))) return true;  // phases complete for good
+    if ((it & 63u) == 0) {
+      int stop = 0;
+      if ((threadIdx.x & 31) == 0) {
+        if (it == 0) {
+          t0 = globaltimer_ns();
+        } else if (*abort_flag) {
+          stop = 1;
+        } else if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          atomicCAS(err, 0, code);
+          *abort_flag = 1;
+          stop = 1;
+        }
+      }
+      if (__shfl_sync(0xffffffffu, stop, 0)) return false;
+    }
+  }
+}
+
 // Warp-uniform bounded wait: lane 0 polls, the result is broadcast.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int* err, int code,
                                           volatile int* abort_flag) {
