@@ -150,13 +150,20 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
     for (int shift = 24; shift >= 0; shift -= 8) {
       for (int it = 0; it < n_iter; ++it) {
         const int j = it * kSelThreads + threadIdx.x;
-        uint32_t digit = 256;
+        // only candidates that still match the prefix are counted; warps with
+        // none (most of them after the first passes) skip the match entirely
+        bool match = false;
+        uint32_t digit = 0;
         if (j < L) {
           const uint32_t u = score_bits(sc[j]);
-          if ((u & pmask) == prefix) digit = (u >> shift) & 255u;
+          match = (u & pmask) == prefix;
+          digit = (u >> shift) & 255u;
         }
-        const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-        if (lane == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
+        const uint32_t act = __ballot_sync(0xffffffffu, match);
+        if (match) {
+          const uint32_t peers = __match_any_sync(act, digit);
+          if (lane == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
+        }
       }
       __syncthreads();
       // suffix counts: warp w < 8 owns bins [32w, 32w+32)
@@ -193,42 +200,39 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
     need_eq = k;
   }
 
-  // 3. keep flags and compaction in pool (= position) order, 512 candidates
-  //    per round: a block-wide scan gives each kept candidate its slot, so
-  //    consecutive threads write consecutive slots (coalesced stores)
-  __shared__ int base_kept, base_eq;
-  if (threadIdx.x == 0) {
-    base_kept = 0;
-    base_eq = 0;
+  // 3. compaction in pool (= position) order with one block-wide scan: thread
+  //    t owns the consecutive candidates [t*C, t*C + C); the scan of its
+  //    (greater, tied) counts gives its first output slot and how many tied
+  //    candidates precede it, so the first need_eq ties in pool order are kept
+  const int C = (L + kSelThreads - 1) / kSelThreads;
+  const int j_lo = min(L, threadIdx.x * C), j_hi = min(L, j_lo + C);
+  uint32_t n_gt = 0, n_eq = 0;
+  for (int j = j_lo; j < j_hi; ++j) {
+    if (keep_all) {
+      ++n_gt;
+    } else {
+      const uint32_t u = score_bits(sc[j]);
+      n_gt += u > tau;
+      n_eq += u == tau;
+    }
   }
-  __syncthreads();
-  for (int j0 = 0; j0 < L; j0 += kSelThreads) {
-    const int j = j0 + threadIdx.x;
-    // kept and tied candidates before this round (read before the scan's barriers)
-    const int bk = base_kept, be = base_eq;
-    uint32_t is_gt = 0, is_eq = 0;
-    if (j < L) {
-      if (keep_all) {
-        is_gt = 1;
-      } else {
-        const uint32_t u = score_bits(sc[j]);
-        is_gt = u > tau;
-        is_eq = u == tau;
-      }
+  const uint32_t packed = block_exclusive_scan(n_gt | (n_eq << 16), warp_tot);
+  int eq_seen = (int)(packed >> 16);                               // tied candidates before j_lo
+  int dst = (int)(packed & 0xffffu) + min(eq_seen, need_eq);       // kept candidates before j_lo
+  int32_t* idx = a.idx + ((long long)s * a.Hkv + G0) * a.B;
+  for (int j = j_lo; j < j_hi; ++j) {
+    bool keep;
+    if (keep_all) {
+      keep = true;
+    } else {
+      const uint32_t u = score_bits(sc[j]);
+      keep = u > tau;
+      if (u == tau) keep = eq_seen++ < need_eq;
     }
-    const uint32_t packed = block_exclusive_scan(is_gt | (is_eq << 16), warp_tot);
-    const int eq_rank = be + (int)(packed >> 16);  // tied candidates before j
-    const bool keep = is_gt || (is_eq && eq_rank < need_eq);
-    const int dst = bk + (int)(packed & 0xffffu) + (min(eq_rank, need_eq) - min(be, need_eq));
-    if (keep && dst < a.B) a.idx[((long long)s * a.Hkv + G0) * a.B + dst] = j;
-    // the last thread of the round holds the round's totals
-    if (threadIdx.x == kSelThreads - 1) {
-      const int gt_all = (int)(packed & 0xffffu) + (int)is_gt;
-      const int eq_all = (int)(packed >> 16) + (int)is_eq;
-      base_kept = bk + gt_all + (min(be + eq_all, need_eq) - min(be, need_eq));
-      base_eq = be + eq_all;
+    if (keep) {
+      if (dst < a.B) idx[dst] = j;
+      ++dst;
     }
-    __syncthreads();
   }
 }
 
