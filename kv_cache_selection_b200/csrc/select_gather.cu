@@ -110,27 +110,70 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
   const float* __restrict__ part = a.part + s * a.part_s;
   const int* __restrict__ pos_c = a.pos_c + ((long long)s * a.Hkv + G0) * a.B;
   const int* __restrict__ pos_f = a.pos_f + (long long)s * a.T;
-  constexpr int kBatch = 4;  // candidates per thread whose loads are in flight together
-  for (int jb = 0; jb < L; jb += kBatch * kSelThreads) {
-    float pv[kBatch][8];
-    int pp[kBatch];
+  if ((a.part_g & 3) == 0 && (reinterpret_cast<uintptr_t>(part) & 15) == 0) {
+    // four consecutive candidates per thread and group as one 16-byte load,
+    // groups summed in the same fixed order
+    const int n4 = (L + 3) / 4;
+    for (int c = threadIdx.x; c < n4; c += kSelThreads) {
+      const int j0 = 4 * c;
+      const bool full = j0 + 3 < L;
+      int pp[4];
 #pragma unroll
-    for (int q = 0; q < kBatch; ++q) {
-      const int j = jb + q * kSelThreads + threadIdx.x;
+      for (int e = 0; e < 4; ++e) {
+        const int j = j0 + e;
+        pp[e] = j < L ? (j < a.m ? __ldg(pos_c + j) : __ldg(pos_f + (j - a.m))) : 0;
+      }
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
-        pv[q][u] = (j < L && G0 + u < G1) ? __ldg(part + (long long)(G0 + u) * a.part_g + j) : 0.f;
-      pp[q] = j < L ? (j < a.m ? __ldg(pos_c + j) : __ldg(pos_f + (j - a.m))) : 0;
+      for (int u = 0; u < 8; ++u) {
+        if (G0 + u < G1) {
+          const float* src = part + (long long)(G0 + u) * a.part_g + j0;
+          float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (full) {
+            x = __ldg(reinterpret_cast<const float4*>(src));
+          } else {
+            x.x = __ldg(src);
+            if (j0 + 1 < L) x.y = __ldg(src + 1);
+            if (j0 + 2 < L) x.z = __ldg(src + 2);
+          }
+          v.x += x.x;
+          v.y += x.y;
+          v.z += x.z;
+          v.w += x.w;
+        }
+      }
+      const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (j0 + e < L) {
+          sc[j0 + e] = vv[e];
+          posp[j0 + e] = pp[e];
+        }
+      }
     }
+  } else {
+    constexpr int kBatch = 4;  // candidates per thread whose loads are in flight together
+    for (int jb = 0; jb < L; jb += kBatch * kSelThreads) {
+      float pv[kBatch][8];
+      int pp[kBatch];
 #pragma unroll
-    for (int q = 0; q < kBatch; ++q) {
-      const int j = jb + q * kSelThreads + threadIdx.x;
-      if (j < L) {
-        float v = 0.f;
+      for (int q = 0; q < kBatch; ++q) {
+        const int j = jb + q * kSelThreads + threadIdx.x;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) v += pv[q][u];
-        sc[j] = v;
-        posp[j] = pp[q];
+        for (int u = 0; u < 8; ++u)
+          pv[q][u] = (j < L && G0 + u < G1) ? __ldg(part + (long long)(G0 + u) * a.part_g + j) : 0.f;
+        pp[q] = j < L ? (j < a.m ? __ldg(pos_c + j) : __ldg(pos_f + (j - a.m))) : 0;
+      }
+#pragma unroll
+      for (int q = 0; q < kBatch; ++q) {
+        const int j = jb + q * kSelThreads + threadIdx.x;
+        if (j < L) {
+          float v = 0.f;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) v += pv[q][u];
+          sc[j] = v;
+          posp[j] = pp[q];
+        }
       }
     }
   }
