@@ -37,6 +37,11 @@ Readings taken where the pages are silent (each is listed in the design doc):
   * "global" selection sums sigma over all query heads and keeps one set for
     every KV head; "per_kv_head" sums over the G query heads of each KV head and
     selects per KV head (P2 §A "Protocol": sinks are kept per layer and KV head);
+  * "recency" is the pages' comparison baseline (P2 Appendix A.3 "Supporting
+    comparison: recency-based retention"; the sliding windows of ReKV in P2's
+    related work): C_n holds the B candidates with the largest positions, i.e.
+    the last B tokens seen, one set for every KV head; scores are computed and
+    reported exactly as in "global" mode but do not decide what is kept;
   * ties are broken by lower original position; C_n is stored in ascending
     original position;
   * while m + T <= B nothing is evicted (top-B of fewer than B candidates);
@@ -64,6 +69,7 @@ MASK_FRAME_CAUSAL = "frame_causal"
 MASK_FRAME_BIDIR = "frame_bidir"
 SELECT_GLOBAL = "global"
 SELECT_PER_KV_HEAD = "per_kv_head"
+SELECT_RECENCY = "recency"
 
 
 def to_f64(x) -> np.ndarray:
@@ -130,6 +136,18 @@ def select_top_b(score: np.ndarray, pos: np.ndarray, B: int) -> np.ndarray:
     else:
         order = np.lexsort((pos, -score))  # primary key: -score, then pos
         kept = order[:B]
+    return kept[np.argsort(pos[kept], kind="stable")]
+
+
+def select_recent_b(pos: np.ndarray, B: int) -> np.ndarray:
+    """Pool indices of the B candidates with the largest positions (the most
+    recent tokens), in ascending position (P2 Appendix A.3: recency-based
+    retention keeps the latest frames of the stream)."""
+    L = pos.shape[0]
+    if L <= B:
+        kept = np.arange(L)
+    else:
+        kept = np.argsort(-pos, kind="stable")[:B]
     return kept[np.argsort(pos[kept], kind="stable")]
 
 
@@ -243,6 +261,11 @@ def statekv_step(state: LayerState, q, k, v, pos, B: int,
         score = np.stack([col_mass[[h for h in range(Hq) if kv_head_of(h, Hq, Hkv) == g]].sum(axis=0)
                           for g in range(Hkv)])
         kept = [select_top_b(score[g], pool_pos[g], B) for g in range(Hkv)]
+    elif select_mode == SELECT_RECENCY:
+        sigma = col_mass.sum(axis=0)
+        score = np.tile(sigma, (Hkv, 1))
+        kept_one = select_recent_b(pool_pos[0], B)
+        kept = [kept_one.copy() for _ in range(Hkv)]
     else:
         raise ValueError(f"unknown select mode {select_mode!r}")
 

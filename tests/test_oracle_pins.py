@@ -124,7 +124,7 @@ def test_zero_budget_is_per_frame_attention():
 
 
 # ------------------------------------------------------ score-mass identity ---
-@pytest.mark.parametrize("select", [O.SELECT_GLOBAL, O.SELECT_PER_KV_HEAD])
+@pytest.mark.parametrize("select", [O.SELECT_GLOBAL, O.SELECT_PER_KV_HEAD, O.SELECT_RECENCY])
 @pytest.mark.parametrize("mask", [O.MASK_FRAME_CAUSAL, O.MASK_FRAME_BIDIR])
 def test_score_mass(select, mask):
     """Each softmax row sums to 1, so the scores of one step sum to Hq*T
@@ -135,7 +135,7 @@ def test_score_mass(select, mask):
     G = Hq // Hkv
     for r in res:
         sums = r["score"].sum(axis=1)
-        want = Hq * T if select == O.SELECT_GLOBAL else G * T
+        want = G * T if select == O.SELECT_PER_KV_HEAD else Hq * T
         np.testing.assert_allclose(sums, want, rtol=1e-13)
 
 
@@ -271,6 +271,50 @@ def test_select_matches_brute_force(seed):
     assert list(got) == _brute_top_b(score, pos, B)
 
 
+# ------------------------------------------------- recency-based retention ---
+def test_recency_keeps_the_last_b_tokens():
+    """Recency retention (P2 Appendix A.3): after frame n, C holds exactly the
+    last min(B, (n+1)T) tokens of the stream, for every KV head, as copies of
+    those tokens' K/V rows."""
+    n_frames, T, Hq, Hkv, d, B = 7, 8, 6, 2, 16, 20
+    frames = random_frames(n_frames, T, Hq, Hkv, d, seed=5)
+    Kall, Vall = concat(frames, 1), concat(frames, 2)
+    st = O.LayerState.empty(Hkv, d)
+    for n, f in enumerate(frames):
+        st, res = O.statekv_step(st, *f, B=B, select_mode=O.SELECT_RECENCY)
+        seen = (n + 1) * T
+        want = np.arange(max(0, seen - B), seen)
+        for g in range(Hkv):
+            np.testing.assert_array_equal(st.pos_C[g], want)
+            np.testing.assert_array_equal(st.K_C[g], Kall[want, g])
+            np.testing.assert_array_equal(st.V_C[g], Vall[want, g])
+
+
+@pytest.mark.parametrize("seed", range(20))
+def test_recency_select_matches_brute_force(seed):
+    """Largest positions first, on pools whose positions arrive in any order."""
+    g = np.random.default_rng(seed)
+    L = int(g.integers(1, 12))
+    B = int(g.integers(0, 12))
+    pos = g.permutation(50)[:L]
+    got = list(O.select_recent_b(pos, B))
+    best = sorted(range(L), key=lambda j: -pos[j])[:B]
+    assert got == sorted(best, key=lambda j: pos[j])
+
+
+def test_recency_changes_only_the_kept_set():
+    """For one and the same state, recency and global steps compute identical
+    attention outputs, row statistics and scores; only C_n differs."""
+    n_frames, T, Hq, Hkv, d, B = 5, 8, 6, 2, 16, 12
+    frames = random_frames(n_frames, T, Hq, Hkv, d, seed=9)
+    st, _ = O.run_stream(frames[:-1], B=B)
+    _, r_g = O.statekv_step(st, *frames[-1], B=B, select_mode=O.SELECT_GLOBAL)
+    _, r_r = O.statekv_step(st, *frames[-1], B=B, select_mode=O.SELECT_RECENCY)
+    for key in ("out", "lse", "score", "pool_pos"):
+        np.testing.assert_array_equal(r_g[key], r_r[key])
+    assert not all(np.array_equal(a, b) for a, b in zip(r_g["kept"], r_r["kept"]))
+
+
 # ------------------------------------------ detailed state and positions ---
 @pytest.mark.parametrize("select", [O.SELECT_GLOBAL, O.SELECT_PER_KV_HEAD])
 def test_detailed_state_is_concatenation(select):
@@ -368,6 +412,13 @@ def _dropped_frame_tokens(mp):
 
 def _wrong_gqa(mp):
     mp.setattr(O, "kv_head_of", lambda h, Hq, Hkv: h % Hkv)   # interleaved groups
+
+
+def test_planted_recency_mistake_is_caught(monkeypatch):
+    """Keeping the oldest instead of the newest tokens fails the recency pin."""
+    monkeypatch.setattr(O, "select_recent_b", lambda pos, B: np.arange(min(B, len(pos))))
+    with pytest.raises(AssertionError):
+        test_recency_keeps_the_last_b_tokens()
 
 
 @pytest.mark.parametrize("patch", [_wrong_mask, _wrong_scale, _wrong_tiebreak,
