@@ -52,8 +52,16 @@ typedef enum { STATEKV_MASK_FRAME_CAUSAL = 0, STATEKV_MASK_FRAME_BIDIR = 1 } sta
 /* Selection granularity.  GLOBAL (default): one score per candidate summed over
  * all query heads, one kept set per layer.  PER_KV_HEAD: scores summed over
  * the query heads of each KV head, a kept set per KV head (P2 Appendix A
- * "Protocol": sinks are kept per layer and KV head). */
-typedef enum { STATEKV_SELECT_GLOBAL = 0, STATEKV_SELECT_PER_KV_HEAD = 1 } statekv_select;
+ * "Protocol": sinks are kept per layer and KV head).  RECENCY: the pages'
+ * comparison baseline (P2 Appendix A.3, recency-based retention): C_n keeps the
+ * B candidates with the largest positions (the last B tokens), one set per
+ * layer; scores are still computed and reported as in GLOBAL mode.  Positions
+ * must be non-negative in this mode. */
+typedef enum {
+  STATEKV_SELECT_GLOBAL = 0,
+  STATEKV_SELECT_PER_KV_HEAD = 1,
+  STATEKV_SELECT_RECENCY = 2
+} statekv_select;
 
 typedef enum {
   STATEKV_OK = 0,
@@ -140,7 +148,8 @@ int statekv_get_detailed(statekv_t h, int layer, const void** k, const void** v,
  *   lse        [S][Hq][T] float32, natural-log log-sum-exp of each query row;
  *   pool_score [S][Hkv][B+T] float32, the score of every pool candidate
  *              (C entries first, then frame tokens); entries [0, pool_len)
- *              valid.  In GLOBAL mode only row 0 of each stream is written.
+ *              valid.  In GLOBAL and RECENCY modes only row 0 of each stream
+ *              is written.
  * Valid until the next prefill_frame.  Any output pointer may be NULL. */
 int statekv_get_step_stats(statekv_t h, const float** lse, const float** pool_score,
                            int* pool_len);

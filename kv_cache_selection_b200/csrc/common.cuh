@@ -101,6 +101,7 @@ struct SelectArgs {
   const int32_t* pos_f;   // frame positions [s][T]
   int32_t* idx;           // out [s][g][B] kept pool indices, ascending (row 0 in global mode)
   int Hkv, m, T, B, global;
+  int recency;            // keep the B largest positions instead of the B largest scores
   int n_sel_blocks;       // blocks [0, n_sel_blocks): one per (stream, selection group)
   // D append: frame [s][t][g][d] -> D [s][g][max_tok][d] at token d_len
   int n_app_blocks;

@@ -179,7 +179,13 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
   }
   for (int b = threadIdx.x; b < 257; b += kSelThreads) hist[b] = 0;
   __syncthreads();
-  for (int j = threadIdx.x; j < L; j += kSelThreads) a.pool_score[s * a.part_s + (long long)G0 * a.part_g + j] = sc[j];
+  for (int j = threadIdx.x; j < L; j += kSelThreads) {
+    a.pool_score[s * a.part_s + (long long)G0 * a.part_g + j] = sc[j];
+    // recency retention ranks by position: the bit pattern of a non-negative
+    // int32 orders like its value, and positions are distinct (no ties)
+    if (a.recency) sc[j] = __int_as_float(max(posp[j], 0));
+  }
+  if (a.recency) __syncthreads();
   if (a.B <= 0) return;  // nothing is kept (block-uniform)
 
   // 2. threshold: the B-th largest score

@@ -120,7 +120,7 @@ int check_shape(statekv_t h, int S, int Hq, int Hkv, int d, int T, int B, int ma
     return set_err(h, STATEKV_ERR_INVALID_ARG, "bad dtype %d", dtype);
   if (mask != STATEKV_MASK_FRAME_CAUSAL && mask != STATEKV_MASK_FRAME_BIDIR)
     return set_err(h, STATEKV_ERR_INVALID_ARG, "bad mask_mode %d", mask);
-  if (select != STATEKV_SELECT_GLOBAL && select != STATEKV_SELECT_PER_KV_HEAD)
+  if (select != STATEKV_SELECT_GLOBAL && select != STATEKV_SELECT_PER_KV_HEAD && select != STATEKV_SELECT_RECENCY)
     return set_err(h, STATEKV_ERR_INVALID_ARG, "bad select_mode %d", select);
   if (d != 64 && d != 128) return set_err(h, STATEKV_ERR_UNSUPPORTED, "head dim %d not in {64,128}", d);
   if ((long long)B + T > 28672)
@@ -542,7 +542,8 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
   se.m = m;
   se.T = T;
   se.B = B;
-  se.global = h->select == STATEKV_SELECT_GLOBAL;
+  se.global = h->select != STATEKV_SELECT_PER_KV_HEAD;  // recency keeps one set per layer too
+  se.recency = h->select == STATEKV_SELECT_RECENCY;
   se.kf = k;
   se.vf = v;
   se.kd = L->kd;

@@ -57,7 +57,8 @@ extern "C" int statekv_step_noalloc(int Hq, int Hkv, int d, int T, int B, int dt
   if (dtype != STATEKV_BF16 && dtype != STATEKV_F32) return fail(STATEKV_ERR_INVALID_ARG, "bad dtype %d", dtype);
   if (mask_mode != STATEKV_MASK_FRAME_CAUSAL && mask_mode != STATEKV_MASK_FRAME_BIDIR)
     return fail(STATEKV_ERR_INVALID_ARG, "bad mask_mode %d", mask_mode);
-  if (select_mode != STATEKV_SELECT_GLOBAL && select_mode != STATEKV_SELECT_PER_KV_HEAD)
+  if (select_mode != STATEKV_SELECT_GLOBAL && select_mode != STATEKV_SELECT_PER_KV_HEAD &&
+      select_mode != STATEKV_SELECT_RECENCY)
     return fail(STATEKV_ERR_INVALID_ARG, "bad select_mode %d", select_mode);
   if (m < 0 || m > B) return fail(STATEKV_ERR_INVALID_ARG, "C length m=%d outside [0, B=%d]", m, B);
   if (d_len < 0 || (long long)d_len + T > max_tok)
@@ -107,7 +108,7 @@ extern "C" int statekv_step_noalloc(int Hq, int Hkv, int d, int T, int B, int dt
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const float scale_log2 = skv::kLog2e / sqrtf((float)d);
   const int causal = mask_mode == STATEKV_MASK_FRAME_CAUSAL;
-  const int global = select_mode == STATEKV_SELECT_GLOBAL;
+  const int global = select_mode != STATEKV_SELECT_PER_KV_HEAD;
   const int m_new = m + T < B ? m + T : B;
 
   skv::AttnArgs aa{};
@@ -173,6 +174,7 @@ extern "C" int statekv_step_noalloc(int Hq, int Hkv, int d, int T, int B, int dt
   se.T = T;
   se.B = B;
   se.global = global;
+  se.recency = select_mode == STATEKV_SELECT_RECENCY;
   se.kf = k;
   se.vf = v;
   se.kd = kd;

@@ -19,7 +19,7 @@ LIB_PATH = os.environ.get("STATEKV_LIB", os.path.join(_PKG, "lib", "libstatekv.s
 
 BF16, F32 = 0, 1
 MASKS = {"frame_causal": 0, "frame_bidir": 1}
-SELECTS = {"global": 0, "per_kv_head": 1}
+SELECTS = {"global": 0, "per_kv_head": 1, "recency": 2}
 N_STAGES = 8
 STAGES = ["attention", "attention_combine", "score", "select", "gather", None, None, None]
 ERRORS = {0: "OK", -1: "INVALID_ARG", -2: "UNSUPPORTED", -3: "CAPACITY", -4: "OOM", -5: "CUDA"}

@@ -36,9 +36,10 @@ def run_stream_parity(wl, n_frames, check, B=None, mask="frame_causal", select="
     h = S.StateKV(wl.Hq, wl.Hkv, wl.d, wl.T, B, max_frames=n_frames, dtype=wl.dtype,
                   mask=mask, select=select, n_streams=n_streams)
     omask = O.MASK_FRAME_CAUSAL if mask == "frame_causal" else O.MASK_FRAME_BIDIR
-    osel = O.SELECT_GLOBAL if select == "global" else O.SELECT_PER_KV_HEAD
+    osel = {"global": O.SELECT_GLOBAL, "per_kv_head": O.SELECT_PER_KV_HEAD, "recency": O.SELECT_RECENCY}[select]
+    per_head = select == "per_kv_head"
     G = wl.Hq // wl.Hkv
-    mass = wl.Hq * wl.T if select == "global" else G * wl.T
+    mass = G * wl.T if per_head else wl.Hq * wl.T
     all_frames = [[Syn.gen_frame(wl, n, layer=layer, stream=s) for s in range(n_streams)]
                   for n in range(n_frames)]
     report = dict(near_boundary=0, checked=0, max_rel_l2=0.0, max_score_rel=0.0)
@@ -66,14 +67,17 @@ def run_stream_parity(wl, n_frames, check, B=None, mask="frame_causal", select="
             P.check_lse(stats["lse"][s], res["lse"], wl.dtype)
             L = stats["pool_len"]
             assert L == st.m + wl.T
-            rows = slice(0, 1) if select == "global" else slice(0, wl.Hkv)
+            rows = slice(0, wl.Hkv) if per_head else slice(0, 1)
             sr = P.check_scores(stats["pool_score"][s, rows, :L], res["score"][rows], mass)
             report["max_score_rel"] = max(report["max_score_rel"], sr)
             assert C_after["len"] == min(B, st.m + wl.T)
             for g in range(wl.Hkv):
                 got_pos = C_after["pos"][s, g, :C_after["len"]].cpu().numpy()
-                report["near_boundary"] += P.check_selection(
-                    got_pos, res["kept"][g], res["score"][g], res["pool_pos"][g], B)
+                if select == "recency":   # positions decide: exact
+                    np.testing.assert_array_equal(got_pos, res["pool_pos"][g][res["kept"][g]])
+                else:
+                    report["near_boundary"] += P.check_selection(
+                        got_pos, res["kept"][g], res["score"][g], res["pool_pos"][g], B)
                 # kept rows are bit-exact copies of the source tokens
                 pool_k = np.concatenate([st.K_C[g], O.to_f64(ks)[:, g]]) if st.m else O.to_f64(ks)[:, g]
                 pool_v = np.concatenate([st.V_C[g], O.to_f64(vs)[:, g]]) if st.m else O.to_f64(vs)[:, g]
@@ -84,7 +88,7 @@ def run_stream_parity(wl, n_frames, check, B=None, mask="frame_causal", select="
                 # stored scores are the pool scores of the kept candidates
                 got_sc = C_after["score"][s, g, :len(sel)].cpu().numpy()
                 np.testing.assert_array_equal(
-                    got_sc, stats["pool_score"][s, 0 if select == "global" else g, sel].cpu().numpy())
+                    got_sc, stats["pool_score"][s, g if per_head else 0, sel].cpu().numpy())
             report["checked"] += 1
     # D holds every frame token unmodified, in arrival order
     torch.cuda.synchronize()
@@ -133,6 +137,24 @@ def test_modes_small(mask, select):
     wl = Syn.workload("1b_layer", Hq=6, Hkv=2, d=64, T=24, B=40, frames=7, n_sinks=3)
     r = run_stream_parity(wl, wl.frames, check=range(wl.frames), mask=mask, select=select)
     assert r["checked"] == wl.frames
+
+
+@cuda
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_recency_mode_small(dtype):
+    """Recency retention: C after every frame is the last B tokens; the
+    attention, scores and D are checked as in the score-based modes."""
+    wl = Syn.workload("1b_layer", Hq=6, Hkv=2, d=64, T=24, B=40, frames=7, n_sinks=3, dtype=dtype)
+    r = run_stream_parity(wl, wl.frames, check=range(wl.frames), select="recency")
+    assert r["checked"] == wl.frames
+
+
+@cuda
+def test_recency_mode_1b_layer():
+    """1B-class layer shape (B=1024, T=256): C fills at frame 4, then slides."""
+    wl = Syn.workload("1b_layer", frames=8)
+    r = run_stream_parity(wl, wl.frames, check={0, 3, 4, 7}, select="recency")
+    assert r["checked"] == 4
 
 
 @cuda
