@@ -367,7 +367,9 @@ cudaError_t launch_select(const SelectArgs& a_in, int S, cudaStream_t st, bool p
     a.n_mrg_blocks = 0;
   }
   const size_t smem = (size_t)L * (sizeof(float) + sizeof(int));
-  if (smem > 48 * 1024) {
+  // the default 48 KB per block covers static and dynamic shared memory
+  // together; the kernel's static arrays take ~1.2 KB, so opt in well before
+  if (smem > 40 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(select_topb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
