@@ -443,6 +443,48 @@ def run_flatness(args):
     print(json.dumps(rep), flush=True)
 
 
+def run_diagnostics(args):
+    """Appendix-A diagnostics on the synthetic sink recipe (1B-class layer
+    shape): concentration, candidate-pool recall and retention from a
+    no-eviction handle, and the historical mass that the score-based C and the
+    recency C capture at the same budget.  Timing-free report."""
+    import numpy as np
+    from kv_cache_selection_b200 import diagnostics as Dg
+    from kv_cache_selection_b200 import statekv as SKV
+    wl = Syn.workload("1b_layer", frames=args.diag_frames)
+    dev = torch.device("cuda")
+    n_tok = wl.frames * wl.T
+    full = SKV.StateKV(wl.Hq, wl.Hkv, wl.d, wl.T, n_tok, max_frames=wl.frames, dtype=wl.dtype)
+    B = args.diag_b
+    sel = {name: SKV.StateKV(wl.Hq, wl.Hkv, wl.d, wl.T, B, max_frames=wl.frames, dtype=wl.dtype, select=mode)
+           for name, mode in (("statekv", "global"), ("recency", "recency"))}
+    steps, kept = [], {name: [] for name in sel}
+    for n in range(wl.frames):
+        q, k, v, pos = (t.to(dev) for t in Syn.gen_frame(wl, n))
+        C = full.get_compressed(0) if n > 0 else None
+        hist_pos = C["pos"][0, 0, :C["len"]].cpu().numpy() if C is not None else np.zeros(0, np.int32)
+        for name, h in sel.items():
+            Cs = h.get_compressed(0) if n > 0 else None
+            kept[name].append(Cs["pos"][0, 0, :Cs["len"]].cpu().numpy().copy() if Cs is not None else None)
+            h.prefill_frame(0, q, k, v, pos)
+        full.prefill_frame(0, q, k, v, pos)
+        torch.cuda.synchronize()
+        stats = full.step_stats()
+        L = stats["pool_len"]
+        steps.append(dict(pos=np.concatenate([hist_pos, pos.cpu().numpy()]).astype(np.int64),
+                          mass=stats["pool_score"][0, 0, :L].double().cpu().numpy(),
+                          frame_pos=pos.cpu().numpy().astype(np.int64)))
+    rep = Dg.stream_report(steps, budgets=args.diag_budgets, retained=kept)
+    out = {"report": "diagnostics", "workload": f"1b_layer shape, {wl.frames} frames, sinks recipe",
+           "budget_of_retained_sets": B,
+           "concentration": rep["concentration"], "weighted_pool_recall": rep["weighted_recall"],
+           "pool_recall": rep["recall"], "retention": rep["retention"],
+           "captured_historical_mass": rep["captured"]}
+    for h in list(sel.values()) + [full]:
+        h.close()
+    print(json.dumps(out), flush=True)
+
+
 def run_stack(args):
     """28 independent 8B-class layers, layers in order per frame, 128 frames."""
     from kv_cache_selection_b200 import statekv as SKV
@@ -611,9 +653,12 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle time")
-    ap.add_argument("--mode", choices=["headline", "flatness", "stack", "sweep"], default="headline",
+    ap.add_argument("--mode", choices=["headline", "flatness", "stack", "sweep", "diagnostics"], default="headline",
                     help="headline: the contract's JSON line; others: report lines")
     ap.add_argument("--stack-frames", type=int, default=0)
+    ap.add_argument("--diag-frames", type=int, default=64)
+    ap.add_argument("--diag-b", type=int, default=1024, help="budget of the retained sets compared")
+    ap.add_argument("--diag-budgets", type=int, nargs="+", default=[1, 16, 256, 1024, 4096])
     ap.add_argument("--sweep-frames", type=int, nargs="+", default=[32, 64, 128, 256, 512, 1024])
     ap.add_argument("--sweep-b", type=int, nargs="+", default=[1024, 2048, 4096])
     args = ap.parse_args(argv)
@@ -621,7 +666,8 @@ def main(argv=None):
         ap.error("--warmup must be >= 3")
     wl = Syn.workload(args.workload)
     if args.mode != "headline":
-        {"flatness": run_flatness, "stack": run_stack, "sweep": run_sweep}[args.mode](args)
+        {"flatness": run_flatness, "stack": run_stack, "sweep": run_sweep,
+         "diagnostics": run_diagnostics}[args.mode](args)
         return
     if args.impl == "reference":
         run_reference(args, wl)
