@@ -59,6 +59,15 @@ def test_host_side_argument_errors():
     # full_causal_prefill argument checks
     assert S.lib.full_causal_prefill(None, None, None, 4, 2, 1, 64, 0, None, None, None) == -1
     assert S.lib.statekv_frames(None, 0) == 0
+    # select modes: 3 does not exist; 2 (recency retention) passes the host checks
+    assert S.lib.statekv_create(ctypes.byref(h), 2, 1, 64, 16, 32, 8, 0, 0, 3) == -1
+    assert b"select" in S.lib.statekv_last_error(None)
+    h2 = ctypes.c_void_p()
+    rc = S.lib.statekv_create(ctypes.byref(h2), 2, 1, 64, 16, 32, 8, 0, 0, 2)
+    assert rc != -1, S.lib.statekv_last_error(None)
+    if rc == 0:
+        S.lib.statekv_destroy(h2)
+    assert S.SELECTS == {"global": 0, "per_kv_head": 1, "recency": 2}
 
 
 def test_binding_refuses_missing_library(tmp_path, monkeypatch):
