@@ -310,3 +310,13 @@ def test_8b_sweep_shape_four_streams():
     wl = Syn.workload("8b_sweep", B=1024, frames=6)
     r = run_stream_parity(wl, wl.frames, check={0, 4, 5}, n_streams=4)
     assert r["checked"] == 3 * 4  # three frames, four streams
+
+
+@cuda
+def test_pool_above_48kb_of_selection_smem():
+    """Pools whose selection needs 46 KB and 48 KB of dynamic shared memory (plus
+    the kernel's static arrays, past the default 48 KB per block): B = 5888 at
+    T = 256 gives pools of 5888 and 6144 candidates at frames 22 and 23."""
+    wl = Syn.workload("1b_layer", B=5888, frames=24)
+    r = run_stream_parity(wl, wl.frames, check={22, 23})
+    assert r["checked"] == 2
