@@ -325,6 +325,38 @@ def causal_attention(q, k, v):
     return out, lse
 
 
+def decode_attention(D_K, D_V, q, k, v):
+    """Attention of n text tokens that follow the video, over the detailed state.
+
+    The detailed state D keeps every frame's K/V for the final generation
+    (P1 §方法步骤详情: the frame's KV go to the detailed cache; P2 related work:
+    the second cache preserves full per-frame visual detail for generation).
+    Text token i sees every retained video token and text tokens 0..i.
+    D_K, D_V [Hkv][N][d]; q [n][Hq][d]; k, v [n][Hkv][d].  Returns
+    out [n][Hq][d], lse [Hq][n] (natural log).
+    """
+    D_K = to_f64(D_K)
+    D_V = to_f64(D_V)
+    q = to_f64(q)
+    k = to_f64(k)
+    v = to_f64(v)
+    n, Hq, d = q.shape
+    Hkv = k.shape[1]
+    N = D_K.shape[1]
+    vis = np.ones((n, N + n), dtype=bool)
+    vis[:, N:] = np.tril(np.ones((n, n), dtype=bool))
+    out = np.zeros((n, Hq, d))
+    lse = np.zeros((Hq, n))
+    for h in range(Hq):
+        g = kv_head_of(h, Hq, Hkv)
+        K_pool = np.concatenate([D_K[g], k[:, g]], axis=0)
+        V_pool = np.concatenate([D_V[g], v[:, g]], axis=0)
+        o_h, lse_h, _ = attend_pool(q[:, h], K_pool, V_pool, vis)
+        out[:, h] = o_h
+        lse[h] = lse_h
+    return out, lse
+
+
 def causal_attention_rows(q, k, v, rows):
     """Causal attention for selected query tokens only (for large N sampling).
 

@@ -315,6 +315,41 @@ def test_recency_changes_only_the_kept_set():
     assert not all(np.array_equal(a, b) for a, b in zip(r_g["kept"], r_r["kept"]))
 
 
+# ------------------------------------------------ decode over the detailed state ---
+@pytest.mark.parametrize("n_text", [1, 5])
+def test_decode_attention_equals_causal_over_the_whole_sequence(n_text):
+    """Text tokens after the video attend over D (every frame token) and
+    causally over the text: the rows of a library causal attention over the
+    concatenated sequence [video; text]."""
+    n_frames, T, Hq, Hkv, d, B = 4, 6, 6, 2, 16, 8
+    frames = random_frames(n_frames, T, Hq, Hkv, d, seed=21)
+    st, _ = O.run_stream(frames, B=B)
+    DK, DV, _ = st.detailed()
+    g = np.random.default_rng(22)
+    q = g.standard_normal((n_text, Hq, d))
+    k = g.standard_normal((n_text, Hkv, d))
+    v = g.standard_normal((n_text, Hkv, d))
+    out, lse = O.decode_attention(DK, DV, q, k, v)
+    Qall = np.concatenate([concat(frames, 0), q])
+    Kall = np.concatenate([concat(frames, 1), k])
+    Vall = np.concatenate([concat(frames, 2), v])
+    ref = sdpa_f64(Qall, Kall, Vall, is_causal=True)[-n_text:]
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+    # lse against a direct log-sum-exp of the visible logits of head 0, row 0
+    N = DK.shape[1]
+    s0 = np.concatenate([DK[0], k[:1, 0]]) @ q[0, 0] / math.sqrt(d)
+    np.testing.assert_allclose(lse[0, 0], np.log(np.exp(s0).sum()), rtol=1e-13)
+    assert N == n_frames * T
+
+
+def test_decode_attention_without_video_is_causal_attention():
+    g = np.random.default_rng(23)
+    n, Hq, Hkv, d = 4, 4, 2, 8
+    q, k, v = g.standard_normal((n, Hq, d)), g.standard_normal((n, Hkv, d)), g.standard_normal((n, Hkv, d))
+    out, _ = O.decode_attention(np.zeros((Hkv, 0, d)), np.zeros((Hkv, 0, d)), q, k, v)
+    np.testing.assert_allclose(out, sdpa_f64(q, k, v, is_causal=True), rtol=0, atol=1e-12)
+
+
 # ------------------------------------------ detailed state and positions ---
 @pytest.mark.parametrize("select", [O.SELECT_GLOBAL, O.SELECT_PER_KV_HEAD])
 def test_detailed_state_is_concatenation(select):
