@@ -29,6 +29,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import torch
@@ -87,8 +88,9 @@ class ClockSampler:
 
     def start(self):
         try:
-            out_dir = os.path.join(ROOT, "gpurun_out") if os.path.isdir(os.path.join(ROOT, "gpurun_out")) \
-                else "/tmp"
+            # STATEKV_CLOCKS_DIR keeps the raw samples for inspection; by
+            # default they go to the system temporary directory
+            out_dir = os.environ.get("STATEKV_CLOCKS_DIR") or tempfile.gettempdir()
             self.path = os.path.join(out_dir, f"clocks_rank{self.gpu}_{os.getpid()}.csv")
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(

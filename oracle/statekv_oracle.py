@@ -27,7 +27,7 @@ layer and frame n with compressed state C_{n-1} (m entries per KV head):
      normalised softmax weight P_ij;
   4. the top-B candidates by score become C_n.
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
   * softmax scale 1/sqrt(d);
   * mask: frame token t is visible to frame query i iff t <= i
     ("frame_causal"; the backbone LLM is causal, P1 §自注意力复杂度); all
