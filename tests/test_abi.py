@@ -81,3 +81,29 @@ def test_binding_refuses_missing_library(tmp_path, monkeypatch):
     monkeypatch.delenv("STATEKV_LIB")
     sys.modules.pop("kv_cache_selection_b200.statekv", None)
     importlib.import_module("kv_cache_selection_b200.statekv")
+
+
+def test_noalloc_host_side_errors():
+    """statekv_step_noalloc validates its arguments before any device call, so
+    these refusals need no GPU.  The pointers are never dereferenced."""
+    from kv_cache_selection_b200 import statekv as S
+    p = ctypes.c_void_p(4096)                  # aligned, never touched
+    q = ctypes.c_void_p(4096 + 8)              # misaligned
+    kc, vc = ctypes.c_void_p(8192), ctypes.c_void_p(12288)
+    f = S.lib.statekv_step_noalloc
+
+    def call(Hq=2, Hkv=1, d=64, T=16, B=32, dtype=S.BF16, mask=0, select=0, qp=p, kcp=kc, vcp=vc,
+             kc_new=p, m=0, d_len=0, max_tok=64):
+        return f(Hq, Hkv, d, T, B, dtype, mask, select, qp, p, p, p, kcp, vcp, p, m, p,
+                 kc_new, ctypes.c_void_p(16384), p, p, p, p, p, d_len, max_tok, None)
+
+    assert call(Hq=3, Hkv=2) == -1                       # Hq not a multiple of Hkv
+    assert call(d=96) == -2                              # unsupported head dim
+    assert call(select=3) == -1                          # no such select mode
+    assert call(mask=5) == -1
+    assert call(m=40) == -1                              # C longer than its capacity
+    assert call(d_len=60) == -3                          # D full
+    assert call(qp=q) == -1                              # misaligned tensor
+    assert call(kc_new=kc) == -1                         # C_n over C_{n-1}
+    assert call(Hq=8, Hkv=8, d=128, T=256, B=30000, max_tok=512) == -2   # beyond the fixed scratch
+    assert b"statekv_create" in S.lib.statekv_last_error(None)
