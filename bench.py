@@ -195,7 +195,8 @@ def run_ours(args, wl):
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     K, W = args.steps, args.warmup
     fill = math.ceil(wl.B / wl.T)
-    total_frames = fill + W + 2 * K   # timed pass + per-stage profiling pass
+    n_enq = min(K, 50)
+    total_frames = fill + W + 2 * K + n_enq   # timed pass, per-stage profiling pass, host enqueue pass
     n_distinct = min(total_frames, args.distinct_frames)
     fr_cpu, Q, Kf, Vf = make_frames(wl, n_distinct, rank, dev)
     pos_all = torch.arange(total_frames * wl.T, dtype=torch.int32, device=dev).view(total_frames, wl.T)
@@ -242,56 +243,58 @@ def run_ours(args, wl):
     ms_steps = [a.elapsed_time(b) for a, b in ev]
     value, ms_total = replica_throughput(K, sum(ms_steps), dev)
 
-    # ---- end to end through the host-buffer C-ABI call (pinned host memory)
+    # ---- end to end through the host-buffer C-ABI call (pinned host memory):
+    # every step copies its frame in and its output back inside the timed
+    # region; the K steps are timed as one region (consecutive steps may overlap
+    # their copies with the previous step's kernels, as a streaming caller would)
     e2e = None
     if not args.no_e2e:
-        qh = torch.empty((wl.T, wl.Hq, wl.d), dtype=wl.torch_dtype).pin_memory()
-        kh = torch.empty((wl.T, wl.Hkv, wl.d), dtype=wl.torch_dtype).pin_memory()
-        vh = torch.empty_like(kh).pin_memory()
-        ph = torch.empty((wl.T,), dtype=torch.int32).pin_memory()
-        oh = torch.empty_like(qh).pin_memory()
         he = SKV.StateKV(wl.Hq, wl.Hkv, wl.d, wl.T, wl.B, max_frames=total_frames, dtype=wl.dtype)
         he.reserve_layers(1)
         host_frames = [(f[0].contiguous().pin_memory(), f[1].contiguous().pin_memory(),
                         f[2].contiguous().pin_memory()) for f in fr_cpu]
+        host_pos = torch.arange(total_frames * wl.T, dtype=torch.int32).view(total_frames, wl.T).pin_memory()
+        host_out = [torch.empty((wl.T, wl.Hq, wl.d), dtype=wl.torch_dtype).pin_memory() for _ in range(2)]
 
         def host_step(n):
             i = n % n_distinct
-            qh.copy_(host_frames[i][0])
-            kh.copy_(host_frames[i][1])
-            vh.copy_(host_frames[i][2])
-            ph.copy_(torch.arange(n * wl.T, (n + 1) * wl.T, dtype=torch.int32))
-            he.prefill_frame_host(0, qh, kh, vh, ph, oh)
+            he.prefill_frame_host(0, host_frames[i][0], host_frames[i][1], host_frames[i][2], host_pos[n],
+                                  host_out[n & 1])
 
         for n in range(fill + W):
             host_step(n)
         torch.cuda.synchronize()
-        ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if world > 1:
             torch.distributed.barrier()
         torch.cuda.synchronize()
+        e0.record()
         for j in range(K):
-            if flush is not None:
-                flush.fill_(j)
-            torch.cuda.current_stream().synchronize()   # host buffers are refilled per step
-            n = fill + W + j
-            i = n % n_distinct
-            qh.copy_(host_frames[i][0])
-            kh.copy_(host_frames[i][1])
-            vh.copy_(host_frames[i][2])
-            ph.copy_(torch.arange(n * wl.T, (n + 1) * wl.T, dtype=torch.int32))
-            ev2[j][0].record()
-            he.prefill_frame_host(0, qh, kh, vh, ph, oh)
-            ev2[j][1].record()
+            host_step(fill + W + j)
+        e1.record()
         torch.cuda.synchronize()
-        e2e_value, e2e_ms = replica_throughput(K, sum(a.elapsed_time(b) for a, b in ev2), dev)
+        e2e_value, e2e_ms = replica_throughput(K, e0.elapsed_time(e1), dev)
         esize = 2 if wl.dtype == "bf16" else 4
         h2d = (wl.T * wl.Hq * wl.d + 2 * wl.T * wl.Hkv * wl.d) * esize + wl.T * 4
         d2h = wl.T * wl.Hq * wl.d * esize
         e2e = {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K,
-               "path": "statekv_prefill_frame_host (pinned host buffers, copies on the step's stream)"}
+               "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / K, 5),
+               "path": "statekv_prefill_frame_host (pinned host buffers; the library stages the copies)",
+               "l2": "not flushed (host copies dominate)"}
         he.close()
+
+    # ---- host enqueue cost of one step (back-to-back calls, no synchronisation)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for j in range(n_enq):
+        step(fill + W + 2 * K + j)
+    host_enqueue_us = (time.perf_counter() - t0) / n_enq * 1e6
+    torch.cuda.synchronize()
+
+    # ---- flatness: the full 512-frame stream of the 8B layer, per-frame time
+    flat = None
+    if not args.no_flatness and wl.name == "8b_layer":
+        flat = flatness_report(SKV, wl, dev)
 
     if rank != 0:
         h.close()
@@ -353,7 +356,8 @@ def run_ours(args, wl):
         "step_us_p50": round(statistics.median(ms_steps) * 1e3, 2),
         "step_us_p99": round(sorted(ms_steps)[int(0.99 * (len(ms_steps) - 1))] * 1e3, 2),
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
-        "gpu_launches_per_step": launches / K, "clocks": clk,
+        "gpu_launches_per_step": launches / K, "host_enqueue_us_per_step": round(host_enqueue_us, 2),
+        "clocks": clk, "flatness": flat,
     }
     print(json.dumps(line), flush=True)
 
@@ -425,24 +429,36 @@ def _flatness(us, first):
             "slope_over_512_frames_pct": round(100 * slope * 512 / p50, 2)}
 
 
-def run_flatness(args):
-    """8B-class layer over all 512 frames: per-frame latency vs frame index."""
-    from kv_cache_selection_b200 import statekv as SKV
+def flatness_report(SKV, wl, dev):
+    """The whole 512-frame stream of the 8B-class layer from an empty state:
+    device time of every frame (CUDA events, L2 flushed between frames), the
+    least-squares slope over the steady state and its p99/p50, with the SM
+    clocks sampled while it runs."""
     wl = Syn.workload("8b_layer")
-    dev = torch.device("cuda")
     q, k, v, pos = Syn.gen_frames_device(wl, wl.frames, device=dev)
-    h = SKV.StateKV(wl.Hq, wl.Hkv, wl.d, wl.T, wl.B, max_frames=wl.frames + 8, dtype=wl.dtype)
+    h = SKV.StateKV(wl.Hq, wl.Hkv, wl.d, wl.T, wl.B, max_frames=wl.frames, dtype=wl.dtype)
     h.reserve_layers(1)
     out = torch.empty_like(q[0])
     flush = torch.empty(64 * 1024 * 1024, dtype=torch.int32, device=dev)
+    clocks = ClockSampler(dev.index or 0)
+    clocks.start()
     us = _per_frame_times(lambda n: h.prefill_frame(0, q[n], k[n], v[n], pos[n], out), wl.frames, flush, dev)
+    clk = clocks.stop()
     fill = math.ceil(wl.B / wl.T)
-    rep = {"report": "flatness", "workload": "8b_layer (512 frames, B=4096), device-drawn synthetic frames",
+    rep = {"workload": "8b_layer: 512 frames from an empty state, B=4096, device-drawn synthetic frames",
            "l2": "flushed between frames", "fill_frames": fill,
            "fill_us": [round(x, 1) for x in us[:fill]], "steady": _flatness(us, fill),
-           "per_frame_us_every_32": [round(x, 1) for x in us[::32]]}
+           "per_frame_us_every_32": [round(x, 1) for x in us[::32]], "clocks": clk}
     h.close()
-    print(json.dumps(rep), flush=True)
+    del q, k, v, pos
+    return rep
+
+
+def run_flatness(args):
+    """8B-class layer over all 512 frames: per-frame latency vs frame index."""
+    from kv_cache_selection_b200 import statekv as SKV
+    rep = flatness_report(SKV, Syn.workload("8b_layer"), torch.device("cuda"))
+    return dict(report="flatness", **rep)
 
 
 def run_diagnostics(args):
@@ -484,7 +500,7 @@ def run_diagnostics(args):
            "captured_historical_mass": rep["captured"]}
     for h in list(sel.values()) + [full]:
         h.close()
-    print(json.dumps(out), flush=True)
+    return out
 
 
 def run_stack(args):
@@ -513,7 +529,7 @@ def run_stack(args):
            "detailed_state_bytes_K_plus_V": d_bytes,
            "per_frame_us_every_8": [round(x, 1) for x in us[::8]]}
     h.close()
-    print(json.dumps(rep), flush=True)
+    return rep
 
 
 def run_sweep(args):
@@ -586,7 +602,7 @@ def run_sweep(args):
         res["crossover_frames"][B] = cross
         res["analytic_crossover_frames_3_passes"][B] = round(3 * (B + wl.T / 2) / wl.T, 1)
         h.close()
-    print(json.dumps(res), flush=True)
+    return res
 
 
 # ------------------------------------------------------------ reference arm --
@@ -654,6 +670,7 @@ def main(argv=None):
                     help="distinct synthetic frames kept on the device (cycled)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-flatness", action="store_true", help="skip the 512-frame flatness pass")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle time")
     ap.add_argument("--mode", choices=["headline", "flatness", "stack", "sweep", "diagnostics"], default="headline",
                     help="headline: the contract's JSON line; others: report lines")
@@ -668,8 +685,12 @@ def main(argv=None):
         ap.error("--warmup must be >= 3")
     wl = Syn.workload(args.workload)
     if args.mode != "headline":
-        {"flatness": run_flatness, "stack": run_stack, "sweep": run_sweep,
-         "diagnostics": run_diagnostics}[args.mode](args)
+        clocks = ClockSampler(0)
+        clocks.start()
+        rep = {"flatness": run_flatness, "stack": run_stack, "sweep": run_sweep,
+               "diagnostics": run_diagnostics}[args.mode](args)
+        rep["clocks"] = clocks.stop()
+        print(json.dumps(rep), flush=True)
         return
     if args.impl == "reference":
         run_reference(args, wl)

@@ -218,6 +218,14 @@ int full_causal_prefill_batched(const void* q, const void* k, const void* v, int
  * own pool, or a latency-critical loop that cannot afford cudaMalloc's
  * implicit device-wide synchronisation.
  *
+ * Arithmetic: for both element types the attention and score passes run on
+ * the CUDA cores (float32 FMA), not on the tensor cores that
+ * statekv_prefill_frame uses for bf16.  bf16 results therefore agree with
+ * statekv_prefill_frame within the parity tolerances, not bit for bit (a
+ * candidate within 1e-4 relative of the B-th score may be kept by one and
+ * not the other), and at the 8B-class shape this entry point is many times
+ * slower; it is not the timed path.
+ *
  * The caller owns every tensor (device pointers, 16-byte aligned):
  *   q [T][Hq][d], k,v [T][Hkv][d], pos [T]        the frame (as prefill_frame);
  *   kc,vc [Hkv][B][d], posc [Hkv][B], m            C_{n-1}: its first m rows;
@@ -227,6 +235,9 @@ int full_causal_prefill_batched(const void* q, const void* k, const void* v, int
  *                                                  not alias kc/vc;
  *   kd,vd [Hkv][max_tok][d], posd [max_tok]        D; the frame is appended at
  *                                                  token d_len (d_len+T <= max_tok).
+ * pos, posc, posc_new, scorec_new and posd need 4-byte alignment.  Every
+ * output range (out, C_n, D) must be disjoint from every input range and from
+ * the other outputs; overlapping buffers are refused with INVALID_ARG.
  * Per-step scratch lives in one file-scope device array of 1 MiB per device
  * (lse [Hq][T], partial and pool scores [Hkv][B+T], kept list [Hkv][B], each
  * rounded up to 256 bytes); shapes that need more are rejected with

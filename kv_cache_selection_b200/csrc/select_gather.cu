@@ -124,10 +124,12 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
         pp[e] = j < L ? (j < a.m ? __ldg(pos_c + j) : __ldg(pos_f + (j - a.m))) : 0;
       }
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      // groups in ascending order, eight loads in flight per chunk
+      for (int gb = G0; gb < G1; gb += 8) {
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        if (G0 + u < G1) {
-          const float* src = part + (long long)(G0 + u) * a.part_g + j0;
+        if (gb + u < G1) {
+          const float* src = part + (long long)(gb + u) * a.part_g + j0;
           float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
           if (full) {
             x = __ldg(reinterpret_cast<const float4*>(src));
@@ -142,6 +144,7 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
           v.w += x.w;
         }
       }
+      }
       const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -154,24 +157,33 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
   } else {
     constexpr int kBatch = 4;  // candidates per thread whose loads are in flight together
     for (int jb = 0; jb < L; jb += kBatch * kSelThreads) {
-      float pv[kBatch][8];
+      float acc[kBatch] = {};
       int pp[kBatch];
 #pragma unroll
       for (int q = 0; q < kBatch; ++q) {
         const int j = jb + q * kSelThreads + threadIdx.x;
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          pv[q][u] = (j < L && G0 + u < G1) ? __ldg(part + (long long)(G0 + u) * a.part_g + j) : 0.f;
         pp[q] = j < L ? (j < a.m ? __ldg(pos_c + j) : __ldg(pos_f + (j - a.m))) : 0;
+      }
+      // groups in ascending order, eight per chunk with their loads in flight
+      for (int gb = G0; gb < G1; gb += 8) {
+        float pv[kBatch][8];
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+          const int j = jb + q * kSelThreads + threadIdx.x;
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            pv[q][u] = (j < L && gb + u < G1) ? __ldg(part + (long long)(gb + u) * a.part_g + j) : 0.f;
+        }
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q)
+#pragma unroll
+          for (int u = 0; u < 8; ++u) acc[q] += pv[q][u];
       }
 #pragma unroll
       for (int q = 0; q < kBatch; ++q) {
         const int j = jb + q * kSelThreads + threadIdx.x;
         if (j < L) {
-          float v = 0.f;
-#pragma unroll
-          for (int u = 0; u < 8; ++u) v += pv[q][u];
-          sc[j] = v;
+          sc[j] = acc[q];
           posp[j] = pp[q];
         }
       }

@@ -63,15 +63,6 @@ extern "C" int statekv_step_noalloc(int Hq, int Hkv, int d, int T, int B, int dt
   if (m < 0 || m > B) return fail(STATEKV_ERR_INVALID_ARG, "C length m=%d outside [0, B=%d]", m, B);
   if (d_len < 0 || (long long)d_len + T > max_tok)
     return fail(STATEKV_ERR_CAPACITY, "D holds %d tokens; appending %d at %d does not fit", max_tok, T, d_len);
-  if (!q || !k || !v || !pos || !out || !kc || !vc || !posc || !kc_new || !vc_new || !posc_new ||
-      !scorec_new || !kd || !vd || !posd)
-    return fail(STATEKV_ERR_INVALID_ARG, "null pointer argument");
-  if (((uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)out | (uintptr_t)kc | (uintptr_t)vc |
-       (uintptr_t)kc_new | (uintptr_t)vc_new | (uintptr_t)kd | (uintptr_t)vd) & 15)
-    return fail(STATEKV_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
-  if (kc == kc_new || vc == vc_new)
-    return fail(STATEKV_ERR_INVALID_ARG, "C_n must not overwrite C_{n-1} (pass a second buffer)");
-
   // scratch carve-up: lse [Hq][T], partial and pool scores [Hkv][B+T], kept [Hkv][B]
   const size_t pool = (size_t)B + T;
   const size_t lse_b = round256((size_t)Hq * T * 4);
@@ -82,6 +73,45 @@ extern "C" int statekv_step_noalloc(int Hq, int Hkv, int d, int T, int B, int dt
     return fail(STATEKV_ERR_UNSUPPORTED,
                 "shape needs %zu bytes of step scratch; statekv_step_noalloc has %zu (use statekv_create)",
                 need, kNoAllocScratchBytes);
+
+  if (!q || !k || !v || !pos || !out || !kc || !vc || !posc || !kc_new || !vc_new || !posc_new ||
+      !scorec_new || !kd || !vd || !posd)
+    return fail(STATEKV_ERR_INVALID_ARG, "null pointer argument");
+  if (((uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)out | (uintptr_t)kc | (uintptr_t)vc |
+       (uintptr_t)kc_new | (uintptr_t)vc_new | (uintptr_t)kd | (uintptr_t)vd) & 15)
+    return fail(STATEKV_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if (((uintptr_t)pos | (uintptr_t)posc | (uintptr_t)posc_new | (uintptr_t)scorec_new | (uintptr_t)posd) & 3)
+    return fail(STATEKV_ERR_INVALID_ARG, "position and score pointers must be 4-byte aligned");
+
+  // Every output range must be disjoint from every input range and from the
+  // other outputs: the kernels read C_{n-1} and the frame while they write C_n
+  // (another thread's row may be overwritten before it is read).  D is read
+  // only in its appended region, which is an output.
+  const size_t es = dtype == STATEKV_BF16 ? 2 : 4;
+  const size_t cb = (size_t)Hkv * B * d * es, ci = (size_t)Hkv * B * 4;
+  const size_t qb = (size_t)T * Hq * d * es, kb = (size_t)T * Hkv * d * es;
+  const size_t db = (size_t)Hkv * max_tok * d * es, dpb = (size_t)max_tok * 4;
+  struct Range {
+    const void* p;
+    size_t n;
+    const char* name;
+  };
+  const Range outs[] = {{out, qb, "out"}, {kc_new, cb, "kc_new"}, {vc_new, cb, "vc_new"},
+                        {posc_new, ci, "posc_new"}, {scorec_new, ci, "scorec_new"},
+                        {kd, db, "kd"}, {vd, db, "vd"}, {posd, dpb, "posd"}};
+  const Range ins[] = {{q, qb, "q"}, {k, kb, "k"}, {v, kb, "v"}, {pos, (size_t)T * 4, "pos"},
+                       {kc, cb, "kc"}, {vc, cb, "vc"}, {posc, ci, "posc"}};
+  auto overlap = [](const Range& x, const Range& y) {
+    const uintptr_t a0 = (uintptr_t)x.p, b0 = (uintptr_t)y.p;
+    return x.n > 0 && y.n > 0 && a0 < b0 + y.n && b0 < a0 + x.n;
+  };
+  for (const Range& o : outs) {
+    for (const Range& i : ins)
+      if (overlap(o, i)) return fail(STATEKV_ERR_INVALID_ARG, "output %s overlaps input %s", o.name, i.name);
+    for (const Range& o2 : outs)
+      if (&o2 < &o && overlap(o, o2))
+        return fail(STATEKV_ERR_INVALID_ARG, "outputs %s and %s overlap", o2.name, o.name);
+  }
 
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

@@ -93,9 +93,9 @@ def test_noalloc_host_side_errors():
     f = S.lib.statekv_step_noalloc
 
     def call(Hq=2, Hkv=1, d=64, T=16, B=32, dtype=S.BF16, mask=0, select=0, qp=p, kcp=kc, vcp=vc,
-             kc_new=p, m=0, d_len=0, max_tok=64):
-        return f(Hq, Hkv, d, T, B, dtype, mask, select, qp, p, p, p, kcp, vcp, p, m, p,
-                 kc_new, ctypes.c_void_p(16384), p, p, p, p, p, d_len, max_tok, None)
+             kc_new=p, m=0, d_len=0, max_tok=64, posc=p, posc_new=p):
+        return f(Hq, Hkv, d, T, B, dtype, mask, select, qp, p, p, p, kcp, vcp, posc, m, p,
+                 kc_new, ctypes.c_void_p(16384), posc_new, p, p, p, p, d_len, max_tok, None)
 
     assert call(Hq=3, Hkv=2) == -1                       # Hq not a multiple of Hkv
     assert call(d=96) == -2                              # unsupported head dim
@@ -105,5 +105,40 @@ def test_noalloc_host_side_errors():
     assert call(d_len=60) == -3                          # D full
     assert call(qp=q) == -1                              # misaligned tensor
     assert call(kc_new=kc) == -1                         # C_n over C_{n-1}
+    assert call(posc=ctypes.c_void_p(4098)) == -1        # misaligned int32 positions
+    assert b"4-byte" in S.lib.statekv_last_error(None)
     assert call(Hq=8, Hkv=8, d=128, T=256, B=30000, max_tok=512) == -2   # beyond the fixed scratch
     assert b"statekv_create" in S.lib.statekv_last_error(None)
+
+
+def test_noalloc_rejects_overlapping_buffers():
+    """Every output of statekv_step_noalloc must be disjoint from every input
+    and from the other outputs (its kernels read C_{n-1} and the frame while
+    they write C_n).  Checked on the host: the pointers are never touched."""
+    from kv_cache_selection_b200 import statekv as S
+    f = S.lib.statekv_step_noalloc
+    Hq, Hkv, d, T, B, max_tok = 2, 1, 64, 16, 32, 64
+    es = 2
+    sizes = dict(q=T * Hq * d * es, k=T * Hkv * d * es, v=T * Hkv * d * es, pos=T * 4,
+                 kc=Hkv * B * d * es, vc=Hkv * B * d * es, posc=Hkv * B * 4, out=T * Hq * d * es,
+                 kc_new=Hkv * B * d * es, vc_new=Hkv * B * d * es, posc_new=Hkv * B * 4,
+                 scorec_new=Hkv * B * 4, kd=Hkv * max_tok * d * es, vd=Hkv * max_tok * d * es,
+                 posd=max_tok * 4)
+    base, addr = 1 << 20, {}
+    for name, n in sizes.items():          # disjoint, 256-byte aligned fake addresses
+        addr[name] = base
+        base += (n + 255) // 256 * 256
+
+    def call(**over):
+        a = dict(addr, **over)
+        P = {k: ctypes.c_void_p(v) for k, v in a.items()}
+        return f(Hq, Hkv, d, T, B, S.BF16, 0, 0, P["q"], P["k"], P["v"], P["pos"], P["kc"], P["vc"],
+                 P["posc"], 0, P["out"], P["kc_new"], P["vc_new"], P["posc_new"], P["scorec_new"],
+                 P["kd"], P["vd"], P["posd"], 0, max_tok, None)
+
+    for out_name, in_name in (("posc_new", "posc"), ("scorec_new", "posc"), ("out", "q"),
+                              ("kd", "k"), ("posd", "pos"), ("vc_new", "kc_new")):
+        assert call(**{out_name: addr[in_name]}) == -1, (out_name, in_name)
+        assert b"overlap" in S.lib.statekv_last_error(None)
+    # a partial overlap (last bytes of an input) is refused too
+    assert call(posc_new=addr["posc"] + sizes["posc"] - 16) == -1

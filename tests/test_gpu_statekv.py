@@ -28,8 +28,10 @@ def _clone_C(C):
 
 
 def run_stream_parity(wl, n_frames, check, B=None, mask="frame_causal", select="global",
-                      n_streams=1, layer=0):
-    """Run n_frames on the GPU; teacher-forced oracle check at frames in `check`."""
+                      n_streams=1, layer=0, host=False):
+    """Run n_frames on the GPU; teacher-forced oracle check at frames in `check`.
+    host=True drives the step through statekv_prefill_frame_host (pinned host
+    inputs and output, copies enqueued by the library)."""
     S = _skv()
     B = wl.B if B is None else B
     dev = torch.device("cuda")
@@ -50,7 +52,14 @@ def run_stream_parity(wl, n_frames, check, B=None, mask="frame_causal", select="
         q, k, v, pos = stack(0), stack(1), stack(2), stack(3)
         do_check = n in check
         C_before = _clone_C(h.get_compressed(layer)) if (do_check and n > 0) else None
-        out = h.prefill_frame(layer, q, k, v, pos)
+        if host:
+            q, k, v, pos = (t.cpu().pin_memory() for t in (q, k, v, pos))
+            out = torch.empty_like(q).pin_memory()
+            h.prefill_frame_host(layer, q, k, v, pos, out)
+            # the host buffers of this frame are released below: let the copies finish
+            torch.cuda.synchronize()
+        else:
+            out = h.prefill_frame(layer, q, k, v, pos)
         if not do_check:
             continue
         torch.cuda.synchronize()
@@ -320,3 +329,118 @@ def test_pool_above_48kb_of_selection_smem():
     wl = Syn.workload("1b_layer", B=5888, frames=24)
     r = run_stream_parity(wl, wl.frames, check={22, 23})
     assert r["checked"] == 2
+
+
+@cuda
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_host_buffer_entry_parity(dtype):
+    """statekv_prefill_frame_host (the end-to-end path: pinned host buffers,
+    host-to-device copies, the step, the copy of out back) over frames that
+    fill C and then evict, each checked against the oracle."""
+    if dtype == "f32":
+        wl = Syn.workload("tiny")
+    else:
+        wl = Syn.workload("1b_layer", Hq=14, Hkv=2, d=64, T=256, B=512, frames=5)
+    r = run_stream_parity(wl, wl.frames, check=range(wl.frames), host=True)
+    assert r["checked"] == wl.frames
+
+
+@cuda
+@pytest.mark.parametrize("dtype,Hq,Hkv,select", [("f32", 12, 12, "global"), ("bf16", 20, 10, "global"),
+                                                ("bf16", 20, 10, "per_kv_head")])
+def test_more_than_eight_kv_heads(dtype, Hq, Hkv, select):
+    """Global selection sums the partial scores of every KV group, including
+    groups past the eighth."""
+    wl = Syn.workload("1b_layer", Hq=Hq, Hkv=Hkv, d=64, T=24, B=40, frames=5, n_sinks=3, dtype=dtype)
+    r = run_stream_parity(wl, wl.frames, check=range(wl.frames), select=select)
+    assert r["checked"] == wl.frames
+
+
+@cuda
+def test_full_causal_prefill_batched_8b_four_sequences():
+    """full_causal_prefill_batched with four independent sequences of 2048
+    tokens at the 8B layer shape (the launch shape of the crossover sweep), on
+    rows sampled across tiles of every sequence."""
+    S = _skv()
+    wl = Syn.workload("8b_sweep")
+    N = 2048
+    seqs = [Syn.gen_tokens(wl, N, stream=s) for s in range(4)]
+    q, k, v = (torch.stack([sq[i] for sq in seqs]).cuda() for i in range(3))
+    out, lse = S.full_causal_prefill(q, k, v)
+    torch.cuda.synchronize()
+    rows = [0, 1, 127, 128, 255, 256, 1023, 1024, 2046, 2047]
+    for s in range(4):
+        ref_out, ref_lse = O.causal_attention_rows(*seqs[s], rows)
+        P.check_out(out[s, rows], ref_out, "bf16", what=f"sequence {s}")
+        P.check_lse(lse[s][:, rows], ref_lse, "bf16")
+
+
+@cuda
+def test_full_causal_prefill_long_sequence_sampled_rows():
+    """One 65,536-token sequence (256 frames of the 8B layer shape, drawn on
+    the device with the same recipe): sampled rows against the oracle."""
+    S = _skv()
+    wl = Syn.workload("8b_layer")
+    n_frames = 256
+    q, k, v, _ = Syn.gen_frames_device(wl, n_frames, device="cuda")
+    N = n_frames * wl.T
+    q = q.reshape(N, wl.Hq, wl.d).contiguous()
+    k = k.reshape(N, wl.Hkv, wl.d).contiguous()
+    v = v.reshape(N, wl.Hkv, wl.d).contiguous()
+    out, lse = S.full_causal_prefill(q, k, v)
+    torch.cuda.synchronize()
+    rows = [0, 1, 4095, 4096, 32767, 32768, 50001, N - 2, N - 1]
+    qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
+    ref_out, ref_lse = O.causal_attention_rows(qc, kc, vc, rows)
+    P.check_out(out[rows], ref_out, "bf16")
+    P.check_lse(lse[:, rows], ref_lse, "bf16")
+
+
+@cuda
+def test_diagnostics_library_fed_match_oracle_fed():
+    """Appendix-A diagnostics computed from the library's no-eviction pool
+    scores agree with the same diagnostics computed from the oracle's masses on
+    the same frames (1B layer shape, 10 frames); the captured-mass comparison
+    of A.3 uses the retained sets of a score-based and a recency handle."""
+    import numpy as np
+    from kv_cache_selection_b200 import diagnostics as Dg
+    S = _skv()
+    wl = Syn.workload("1b_layer", frames=10)
+    n_tok = wl.frames * wl.T
+    dev = torch.device("cuda")
+    full = S.StateKV(wl.Hq, wl.Hkv, wl.d, wl.T, n_tok, max_frames=wl.frames, dtype=wl.dtype)
+    Bsel = 512
+    sel = {name: S.StateKV(wl.Hq, wl.Hkv, wl.d, wl.T, Bsel, max_frames=wl.frames, dtype=wl.dtype, select=mode)
+           for name, mode in (("statekv", "global"), ("recency", "recency"))}
+    st = O.LayerState.empty(wl.Hkv, wl.d)
+    gpu_steps, ora_steps, kept = [], [], {name: [] for name in sel}
+    for n in range(wl.frames):
+        q, k, v, pos = Syn.gen_frame(wl, n)
+        for name, h in sel.items():
+            Cs = h.get_compressed(0) if n > 0 else None
+            kept[name].append(Cs["pos"][0, 0, :Cs["len"]].cpu().numpy().copy() if Cs is not None else None)
+            h.prefill_frame(0, q.to(dev), k.to(dev), v.to(dev), pos.to(dev))
+        full.prefill_frame(0, q.to(dev), k.to(dev), v.to(dev), pos.to(dev))
+        torch.cuda.synchronize()
+        stats = full.step_stats()
+        L = stats["pool_len"]
+        gmass = stats["pool_score"][0, 0, :L].double().cpu().numpy()
+        st, res = O.statekv_step(st, q, k, v, pos.numpy(), n_tok)
+        assert L == (n + 1) * wl.T
+        P.check_scores(gmass[None], res["score"][:1], wl.Hq * wl.T)
+        fpos = pos.numpy().astype(np.int64)
+        gpu_steps.append(dict(pos=np.arange(L, dtype=np.int64), mass=gmass, frame_pos=fpos))
+        ora_steps.append(dict(pos=res["pool_pos"][0].astype(np.int64), mass=res["score"][0], frame_pos=fpos))
+    budgets = [64, 256, 1024]
+    rg = Dg.stream_report(gpu_steps, budgets, retained=kept)
+    ro = Dg.stream_report(ora_steps, budgets, retained=kept)
+    for B in budgets:
+        # concentration is a sum of masses: close; the set-valued metrics may
+        # differ by a swap at the B-th boundary (1/B each)
+        assert abs(rg["concentration"][B] - ro["concentration"][B]) <= 1e-3
+        for key in ("weighted_recall", "recall", "retention"):
+            assert abs(rg[key][B] - ro[key][B]) <= 2.0 / B + 1e-3, (key, B, rg[key][B], ro[key][B])
+    for name in sel:
+        assert abs(rg["captured"][name] - ro["captured"][name]) <= 1e-3
+    for h in list(sel.values()) + [full]:
+        h.close()

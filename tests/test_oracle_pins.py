@@ -461,3 +461,60 @@ def test_planted_recency_mistake_is_caught(monkeypatch):
                                    _wrong_gqa])
 def test_planted_mistakes_are_caught(monkeypatch, patch):
     assert _pins_fail(monkeypatch, patch)
+
+
+# ------------------------------------- sampled-row causal attention pins ---
+def _rows_pin(Hq=7, Hkv=1, N=300, d=16, seed=11, rows=(0, 1, 2, 127, 128, 129, 255, 256, 298, 299)):
+    """causal_attention_rows at rows that span the first row, 128-token tile
+    boundaries and the last row, against torch SDPA (is_causal) in float64 for
+    out, and for lse against a second SDPA call with one extra "probe" key
+    (zero logit, visible to every row) whose value is a one-hot extra channel:
+    that channel's output is p = 1 / (1 + sum_j exp(s_ij)), so
+    lse_i = log((1 - p) / p).  Also the uniform case q = 0: lse_i = log(i + 1)."""
+    g = np.random.default_rng(seed)
+    q = g.standard_normal((N, Hq, d))
+    k = g.standard_normal((N, Hkv, d))
+    v = g.standard_normal((N, Hkv, d))
+    rows = list(rows)
+    out, lse = O.causal_attention_rows(q, k, v, rows)
+    ref = sdpa_f64(q, k, v, is_causal=True)
+    np.testing.assert_allclose(out, ref[rows], rtol=0, atol=1e-12)
+    # probe-key identity for lse
+    kp = np.concatenate([np.zeros((1, Hkv, d)), k], axis=0)
+    vp = np.concatenate([np.zeros((1, Hkv, d + 1)), np.concatenate([v, np.zeros((N, Hkv, 1))], axis=2)], axis=0)
+    vp[0, :, d] = 1.0
+    mask = torch.ones((N, N + 1), dtype=torch.bool)
+    mask[:, 1:] = torch.tril(torch.ones((N, N), dtype=torch.bool))
+    probe = sdpa_f64(q, kp, vp, attn_mask=mask)[:, :, d]      # [N][Hq]
+    want = np.log((1.0 - probe) / probe).T                    # [Hq][N]
+    np.testing.assert_allclose(lse, want[:, rows], rtol=0, atol=1e-9)
+    # uniform attention: every visible logit is 0
+    _, lse0 = O.causal_attention_rows(np.zeros_like(q), k, v, rows)
+    np.testing.assert_allclose(lse0, np.log(np.asarray(rows, dtype=np.float64) + 1)[None, :].repeat(Hq, 0),
+                               rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(7, 1), (14, 2), (4, 4)])
+def test_causal_attention_rows_pinned(Hq, Hkv):
+    _rows_pin(Hq=Hq, Hkv=Hkv)
+
+
+def test_causal_attention_rows_planted_mistakes(monkeypatch):
+    """Plant an off-by-one in the visible prefix (keys 0..i-1 instead of 0..i)
+    and an interleaved GQA map in the oracle; the pins above must fail."""
+    import inspect
+    import textwrap
+
+    src = textwrap.dedent(inspect.getsource(O.causal_attention_rows))
+    assert src.count("i + 1") == 3
+    bad_src = src.replace("k[:i + 1", "k[:i").replace("v[:i + 1", "v[:i").replace("(1, i + 1)", "(1, i)")
+    ns = dict(O.__dict__)
+    exec(bad_src, ns)
+    monkeypatch.setattr(O, "causal_attention_rows", ns["causal_attention_rows"])
+    # row 0 would see no key at all under this mistake: sample rows >= 1
+    with pytest.raises(AssertionError):
+        _rows_pin(rows=(1, 2, 127, 128, 299))
+    monkeypatch.undo()
+    monkeypatch.setattr(O, "kv_head_of", lambda h, Hq, Hkv: h % Hkv)
+    with pytest.raises(AssertionError):
+        _rows_pin(Hq=14, Hkv=2)
