@@ -292,9 +292,9 @@ def run_ours(args, wl):
     torch.cuda.synchronize()
 
     # ---- flatness: the full 512-frame stream of the 8B layer, per-frame time
-    flat = None
+    flat = dec = None
     if not args.no_flatness and wl.name == "8b_layer":
-        flat = flatness_report(SKV, wl, dev)
+        flat, dec = flatness_report(SKV, wl, dev)
 
     if rank != 0:
         h.close()
@@ -305,6 +305,11 @@ def run_ours(args, wl):
     # ---- roofline of the dominant kernel
     peaks, peak_src = load_peaks()
     work = step_work(wl, wl.B)
+    # the merge of the attention's key splits is part of (a): charge it there
+    if stages.get("attention_combine", (0, 0))[1]:
+        a_ms, a_n = stages["attention"]
+        stages["attention"] = (a_ms + stages["attention_combine"][0], a_n)
+    stages.pop("attention_combine", None)
     stage_us = {k: (v[0] / max(v[1], 1)) * 1e3 for k, v in stages.items() if v[1]}
     dominant = max(stage_us, key=lambda k: stages[k][0])
     bound, amount = work.get(dominant, ("tensor", 0))
@@ -352,12 +357,13 @@ def run_ours(args, wl):
                    "parallelism": f"replicas x{world} (no data-path collective)"},
         "roofline": roofline,
         "stages_us": per_stage,
-        "stages_note": "per-kernel CUDA events in a second pass of K steps (events serialise the kernels)",
+        "stages_note": ("per-kernel CUDA events in a second pass of K steps (events serialise the kernels); "
+                        "attention includes the merge of its key splits, launched on its own in that pass"),
         "step_us_p50": round(statistics.median(ms_steps) * 1e3, 2),
         "step_us_p99": round(sorted(ms_steps)[int(0.99 * (len(ms_steps) - 1))] * 1e3, 2),
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
         "gpu_launches_per_step": launches / K, "host_enqueue_us_per_step": round(host_enqueue_us, 2),
-        "clocks": clk, "flatness": flat,
+        "clocks": clk, "flatness": flat, "decode": dec,
     }
     print(json.dumps(line), flush=True)
 
@@ -449,16 +455,50 @@ def flatness_report(SKV, wl, dev):
            "l2": "flushed between frames", "fill_frames": fill,
            "fill_us": [round(x, 1) for x in us[:fill]], "steady": _flatness(us, fill),
            "per_frame_us_every_32": [round(x, 1) for x in us[::32]], "clocks": clk}
-    h.close()
     del q, k, v, pos
-    return rep
+    dec = decode_report(h, wl, dev, flush)
+    h.close()
+    return rep, dec
+
+
+def decode_report(h, wl, dev, flush, n_texts=(1, 16, 64), reps=5):
+    """Decode attention of n text tokens over the layer's whole detailed state
+    (512 frames = 131,072 tokens): device time per call (CUDA events, L2
+    flushed before each call) against the HBM roofline; the algorithmic bytes
+    are D's K and V read once (2 * Hkv * N * d * 2) plus the text q, k, v, out."""
+    peaks, src = load_peaks()
+    N = h.frames(0) * wl.T
+    res = {"workload": f"8b_layer: decode over D after {h.frames(0)} frames ({N} tokens)", "per_n_text": {}}
+    for n in n_texts:
+        wl_t = Syn.workload(wl.name, T=n, dist="iid", n_sinks=0, drift=0)
+        q, k, v, _ = Syn.gen_frames_device(wl_t, 1, device=dev)
+        q, k, v = q[0], k[0], v[0]
+        out = torch.empty_like(q)
+        h.decode(0, q, k, v, out=out, with_lse=False)   # warm-up (allocates split scratch)
+        ts = []
+        for r in range(reps):
+            flush.fill_(r)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            h.decode(0, q, k, v, out=out, with_lse=False)
+            e1.record()
+            ts.append((e0, e1))
+        torch.cuda.synchronize()
+        us = statistics.median(a.elapsed_time(b) for a, b in ts) * 1e3
+        byts = 2 * wl.Hkv * N * wl.d * 2 + (2 * n * wl.Hq + 2 * n * wl.Hkv) * wl.d * 2
+        gbs = byts / us / 1e3
+        res["per_n_text"][n] = {"us": round(us, 2), "bytes": byts, "gbs": round(gbs, 1),
+                                "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+    res["peak_gbs"] = peaks["hbm_gbs"]
+    res["peak_source"] = f"{src} (copy)"
+    return res
 
 
 def run_flatness(args):
     """8B-class layer over all 512 frames: per-frame latency vs frame index."""
     from kv_cache_selection_b200 import statekv as SKV
-    rep = flatness_report(SKV, Syn.workload("8b_layer"), torch.device("cuda"))
-    return dict(report="flatness", **rep)
+    rep, dec = flatness_report(SKV, Syn.workload("8b_layer"), torch.device("cuda"))
+    return dict(report="flatness", decode=dec, **rep)
 
 
 def run_diagnostics(args):

@@ -116,14 +116,34 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k,
 
 /* statekv_prefill_frame with HOST buffers: q, k, v, pos are read from and out
  * is written to host memory (same layouts; page-locked memory makes the copies
- * asynchronous, pageable memory is accepted).  The call enqueues the
- * host-to-device copies into library-owned staging buffers, the step, and the
- * device-to-host copy of out on `stream`; out is complete once the stream has
- * reached that point (synchronise the stream before reading it).  Calls on one
- * handle reuse the same staging buffers, so successive host calls are ordered
- * by the stream.  Errors: as statekv_prefill_frame. */
+ * asynchronous, pageable memory is accepted).  The call copies the inputs into
+ * one of two library-owned staging sets on a library-owned copy stream (so the
+ * copies of call n+1 overlap the step of call n), makes `stream` wait for them,
+ * enqueues the step and the device-to-host copy of out on `stream`.  When
+ * `stream` has reached the end of the call, the inputs have been read and out
+ * is complete (synchronise the stream before reading out or reusing the input
+ * buffers).  The first call creates the staging buffers, the copy stream and
+ * its events (synchronous).  Errors: as statekv_prefill_frame. */
 int statekv_prefill_frame_host(statekv_t h, int layer, const void* q, const void* k,
                                const void* v, const int32_t* pos, void* out, void* stream);
+
+/* Decode attention over the detailed state D of a layer: the n_text tokens
+ * that follow the video (a question, or generated text) attend to every
+ * video token D holds and causally to each other (P1 section 方法步骤详情: the
+ * frame's KV pairs go to the detailed cache; P2 section 3.2: the second cache
+ * keeps full per-frame detail for the final generation).
+ *   q   [S][n_text][Hq][d]   text queries (device, dtype), RoPE applied
+ *   k,v [S][n_text][Hkv][d]  text keys and values (device, dtype)
+ *   out [S][n_text][Hq][d]   (device, dtype)
+ *   lse [S][Hq][n_text]      float32 natural-log log-sum-exp (device) or NULL
+ * Text token i sees D tokens [0, frames*T) of the layer and text tokens 0..i.
+ * D is read, not modified.  bf16 runs on the tensor cores with the G query
+ * heads of a KV group stacked in one tile, so each D tile crosses HBM once
+ * per KV head; float32 runs on the CUDA cores.  Split scratch is allocated on
+ * the first call that needs more than before (synchronous), then reused.
+ * Errors: INVALID_ARG (unknown layer, bad pointer), OOM, CUDA. */
+int statekv_decode(statekv_t h, int layer, const void* q, const void* k, const void* v, int n_text,
+                   void* out, float* lse, void* stream);
 
 /* Borrow the compressed state C_n of a layer (device pointers owned by the
  * library; valid until the next prefill_frame on that layer or destroy):
@@ -161,13 +181,17 @@ typedef enum {
   STATEKV_STAGE_SCORE = 2,             /* (b) score pass                       */
   STATEKV_STAGE_SELECT = 3,            /* (c) top-B select                     */
   STATEKV_STAGE_GATHER = 4,            /* (d) gather into C_n + append to D    */
+  STATEKV_STAGE_DECODE = 5,            /* statekv_decode attention             */
+  STATEKV_STAGE_DECODE_COMBINE = 6,    /* statekv_decode merge of key splits   */
   STATEKV_N_STAGES = 8
 } statekv_stage;
 
 /* Per-stage device timing: when on, every later prefill_frame records a CUDA
  * event pair around each kernel on the call's stream (a few microseconds of
- * extra enqueue cost; leave off in production).  Turning it off drops
- * unread records. */
+ * extra enqueue cost; leave off in production), and the merge of the
+ * attention's key splits, which otherwise rides in the select launch, runs as
+ * its own launch so that its time is recorded under ATTENTION_COMBINE.
+ * Turning it off drops unread records. */
 int statekv_profile_enable(statekv_t h, int on);
 
 /* Accumulated device time and launch count per stage since the last read:

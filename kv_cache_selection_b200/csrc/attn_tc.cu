@@ -72,15 +72,23 @@ struct TileInfo {
 __device__ __forceinline__ TileInfo tile_info(const AttnTcArgs& a, int g, int t) {
   TileInfo ti;
   const int G = a.Hq / a.Hkv;
-  ti.valid = t < G * a.n_it;
-  if (!ti.valid) t = 0;
-  ti.h = g * G + t / a.n_it;
-  ti.i0 = (t % a.n_it) * 128;
-  int nf = a.nF;
-  if (a.causal) {
-    const int i_max = min(ti.i0 + 127, a.T - 1);  // last row of the tile
-    nf = i_max / 128 + 1;                          // frame tiles holding tokens <= i_max
+  int i_max;
+  if (a.stack) {
+    const int ri = 128 / a.stack;  // rows of the tile per head
+    ti.valid = t < a.n_it;
+    if (!ti.valid) t = 0;
+    ti.h = g * G;                  // first head of the stack
+    ti.i0 = t * ri;
+    i_max = min(ti.i0 + ri - 1, a.T - 1);
+  } else {
+    ti.valid = t < G * a.n_it;
+    if (!ti.valid) t = 0;
+    ti.h = g * G + t / a.n_it;
+    ti.i0 = (t % a.n_it) * 128;
+    i_max = min(ti.i0 + 127, a.T - 1);  // last row of the tile
   }
+  int nf = a.nF;
+  if (a.causal) nf = i_max / 128 + 1;   // frame tiles holding tokens <= i_max
   ti.nk = a.nC + nf;
   return ti;
 }
@@ -162,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const int nq = (nA > 0 ? 1 : 0) + (nB > 0 ? 1 : 0);
       if (nq) {
-        mbar_arrive_expect_tx(bar_q, nq * L::kTileBytes);
+        mbar_arrive_expect_tx(bar_q, nq * L::kAtoms * a.q_rows * 128);
         for (int at = 0; at < L::kAtoms; ++at) {
           if (nA > 0) tma_load_4d(sb + L::kQ + at * L::kAtomBytes, &tm_q, bar_q, at * 64, tA.h, tA.i0, s);
           if (nB > 0)
@@ -264,7 +272,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nX = x == 0 ? nA : nB;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // row within the tile (= TMEM lane)
-    const int i = ti.i0 + r;            // query row in the frame
+    // query row in the frame and query head of this TMEM lane
+    const int i = a.stack ? ti.i0 + r / a.stack : ti.i0 + r;
+    const int h = a.stack ? ti.h + r % a.stack : ti.h;
+    const bool row_exists = !a.stack || r < a.q_rows;
     const uint32_t t_s = tmem + ((uint32_t)(quarter * 32) << 16) + col_s(x);
     const uint32_t t_o = tmem + ((uint32_t)(quarter * 32) << 16) + col_o(x);
     const float c = a.scale_log2;
@@ -353,12 +364,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok && nX > 0) ok = warp_wait(bar_odone(x), 0, a.err, kErrWaitAcc, abort_flag);
     if (ok && ti.valid && !*abort_flag) {
       fence_after_sync();
-      const bool row_ok = i < a.T;
+      const bool row_ok = row_exists && i < a.T;
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const float lse2 = l > 0.f ? m_used + __log2f(l) : -INFINITY;
       if (a.n_split == 1) {
         __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + s * a.out_s + (long long)i * a.out_row +
-                              (long long)ti.h * D;
+                              (long long)h * D;
 #pragma unroll
         for (int c0 = 0; c0 < D / 32; ++c0) {
           uint32_t v[32];
@@ -374,10 +385,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int q4 = 0; q4 < 4; ++q4) dst[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
           }
         }
-        if (row_ok && a.lse) a.lse[s * a.lse_s + (long long)ti.h * a.T + i] = lse2 * kLn2;
+        if (row_ok && a.lse) a.lse[s * a.lse_s + (long long)h * a.T + i] = lse2 * kLn2;
       } else {
-        const long long prow = ((long long)(s * a.Hq + ti.h) * a.n_split + sp) * a.T + i;
-        __nv_bfloat16* orow = a.o_part + prow * D;
+        const long long prow = ((long long)(s * a.Hq + h) * a.n_split + sp) * a.T + i;
 #pragma unroll
         for (int c0 = 0; c0 < D / 32; ++c0) {
           uint32_t v[32];
@@ -388,14 +398,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj) v[jj] = 0u;
           }
-          uint32_t pk[16];
+          if (a.o_part32) {
+            if (row_ok) {
+              float4* dst = reinterpret_cast<float4*>(a.o_part32 + prow * D + c0 * 32);
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj)
-            pk[jj] = pack_bf16x2(__uint_as_float(v[2 * jj]) * inv, __uint_as_float(v[2 * jj + 1]) * inv);
-          if (row_ok) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c0 * 32);
+              for (int q4 = 0; q4 < 8; ++q4)
+                dst[q4] = make_float4(__uint_as_float(v[4 * q4]) * inv, __uint_as_float(v[4 * q4 + 1]) * inv,
+                                      __uint_as_float(v[4 * q4 + 2]) * inv, __uint_as_float(v[4 * q4 + 3]) * inv);
+            }
+          } else {
+            uint32_t pk[16];
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) dst[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+            for (int jj = 0; jj < 16; ++jj)
+              pk[jj] = pack_bf16x2(__uint_as_float(v[2 * jj]) * inv, __uint_as_float(v[2 * jj + 1]) * inv);
+            if (row_ok) {
+              uint4* dst = reinterpret_cast<uint4*>(a.o_part + prow * D + c0 * 32);
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4)
+                dst[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+            }
           }
         }
         if (row_ok) a.ml_part[prow] = nX > 0 ? lse2 : -INFINITY;
@@ -417,7 +438,56 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(MergeArgs a) {
   merge_chunk<D>(a, blockIdx.x * blockDim.x + threadIdx.x);
 }
 
+// Merge of n_split float32 partials (O/l and log2-sum-exp per split): thread
+// = (row, 4-element chunk of d); pass 1 takes the largest log2-sum-exp, pass
+// 2 adds the splits' O/l weighted by 2^(ml_u - max).
+template <int D>
+__global__ void __launch_bounds__(256) attn_merge_wide_kernel(AttnTcArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  constexpr int kChunks = D / 4;
+  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long rows = (long long)a.S * a.Hq * a.T;
+  if (t >= rows * kChunks) return;
+  const int chunk = (int)(t % kChunks);
+  const long long rw = t / kChunks;
+  const int i = (int)(rw % a.T);
+  const long long sh = rw / a.T;  // s * Hq + h
+  const int h = (int)(sh % a.Hq), s = (int)(sh / a.Hq);
+  const long long prow0 = sh * a.n_split * a.T + i;
+  float mx = -INFINITY;
+  for (int u = 0; u < a.n_split; ++u) mx = fmaxf(mx, __ldg(a.ml_part + prow0 + (long long)u * a.T));
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float wsum = 0.f;
+  for (int u = 0; u < a.n_split; ++u) {
+    const float ml = __ldg(a.ml_part + prow0 + (long long)u * a.T);
+    if (ml == -INFINITY) continue;
+    const float w = ex2_approx(ml - mx);
+    const float4 o = __ldg(reinterpret_cast<const float4*>(a.o_part32 + (prow0 + (long long)u * a.T) * D) + chunk);
+    wsum += w;
+    acc.x += w * o.x;
+    acc.y += w * o.y;
+    acc.z += w * o.z;
+    acc.w += w * o.w;
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + s * a.out_s + (long long)i * a.out_row + (long long)h * D;
+  uint2 pk;
+  pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+  pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+  reinterpret_cast<uint2*>(orow)[chunk] = pk;
+  if (chunk == 0 && a.lse)
+    a.lse[s * a.lse_s + (long long)h * a.T + i] = wsum > 0.f ? (mx + __log2f(wsum)) * kLn2 : -INFINITY;
+}
+
 }  // namespace
+
+cudaError_t launch_attn_merge_wide(const AttnTcArgs& a, int d, cudaStream_t st, bool pdl) {
+  const long long rows = (long long)a.S * a.Hq * a.T;
+  const int blocks = (int)((rows * (d / 4) + 255) / 256);
+  if (d == 128) return launch_kernel(attn_merge_wide_kernel<128>, dim3(blocks), dim3(256), 0, st, pdl, a);
+  return launch_kernel(attn_merge_wide_kernel<64>, dim3(blocks), dim3(256), 0, st, pdl, a);
+}
 
 int attn_tc_splits(int S, int Hq, int Hkv, int T, int m, int n_sm) {
   const int G = Hq / Hkv;

@@ -90,39 +90,31 @@ struct MergeArgs {
 };
 
 // Top-B selection over the pool of one (stream, selection group).  The same
-// launch carries extra blocks that append the frame to the detailed state and
-// merge the attention's key-split partials (neither is on the path to C_n).
+// launch carries extra blocks that merge the attention's key-split partials
+// (not on the path to C_n).
 struct SelectArgs {
   const float* part;      // part[s][g][j], j < m + T
   long long part_s;
   int part_g;
   float* pool_score;      // out, same layout as part (row of the selection group only)
-  const int32_t* pos_c;   // current C positions [s][g][B]
-  const int32_t* pos_f;   // frame positions [s][T]
+  const int32_t* pos_c;   // current C positions [s][g][B] (read in recency mode)
+  const int32_t* pos_f;   // frame positions [s][T] (read in recency mode)
   int32_t* idx;           // out [s][g][B] kept pool indices, ascending (row 0 in global mode)
   int Hkv, m, T, B, global;
   int recency;            // keep the B largest positions instead of the B largest scores
   int n_sel_blocks;       // blocks [0, n_sel_blocks): one per (stream, selection group)
-  // D append: frame [s][t][g][d] -> D [s][g][max_tok][d] at token d_len
-  int n_app_blocks;
-  const void* kf;
-  const void* vf;
-  void* kd;
-  void* vd;
-  int32_t* pos_d;         // [s][max_tok]
-  int row_bytes, d_len, max_tok, S;
   // key-split merge (n_mrg_blocks > 0 only for the bf16 attention with splits)
   int n_mrg_blocks;
   MergeArgs mrg;
 };
 
-// Gather of the kept rows into the next C buffer plus the append of the
-// frame's K/V to D.
+// Gather of the kept rows into the next C buffer, plus the append of the
+// frame's K/V and positions to the detailed state D.
 struct GatherArgs {
   const void* kc;  const void* vc;   // current C [s][g][B][d]
   const void* kf;  const void* vf;   // frame [s][t][g][d]
   void* kc_new;    void* vc_new;     // next C [s][g][B][d]
-  const int32_t* idx;                // [s][g][B]
+  const int32_t* idx;                // [s][g][B] kept pool indices (row 0 in global mode)
   void* kd;        void* vd;         // D [s][g][max_tok][d]
   int32_t* pos_d;                    // [s][max_tok]
   const int32_t* pos_f;              // [s][T]

@@ -58,6 +58,12 @@ cudaError_t launch_score_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kc, c
                             const ScoreTcArgs& a, int d, cudaStream_t st, bool pdl = false);
 
 // Tensor-core attention (bf16) over [compressed rows; frame tokens].
+// Query tiles: with stack = 0 a tile is 128 consecutive rows of one query
+// head (n_it tiles per head); with stack = G (the group size) a tile stacks
+// the G query heads of a KV group for 128 / G consecutive rows, row r of the
+// tile being (row i0 + r / G, head g*G + r % G), so every K/V tile is read
+// once for the whole group (n_it tiles per group).  q_rows is the number of
+// rows the Q tensor map's box fills (128, or G * (128 / G)).
 struct AttnTcArgs {
   void* out;          // out[s][i][h][dd] bf16
   long long out_s;
@@ -65,9 +71,11 @@ struct AttnTcArgs {
   float* lse;         // [S][Hq][T] natural log, may be null
   long long lse_s;
   __nv_bfloat16* o_part;  // [S][Hq][n_split][T][d] O/l per split (n_split > 1)
+  float* o_part32;    // same layout in float32; used instead of o_part when set
   float* ml_part;     // [S][Hq][n_split][T] log2-sum-exp
   int m, T, Hq, Hkv, causal, S;
   int n_it, n_pairs, n_split, nC, nF;
+  int stack, q_rows;
   float scale_log2;
   int* err;
 };
@@ -76,6 +84,8 @@ cudaError_t launch_attn_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kc, co
                            const CUtensorMap& tm_kf, const CUtensorMap& tm_vf, const AttnTcArgs& a, int d,
                            cudaStream_t st, bool pdl = false);
 cudaError_t launch_attn_combine(const AttnTcArgs& a, int d, cudaStream_t st, bool pdl = false);
+// Merge of any number of float32 key-split partials (o_part32) into out and lse.
+cudaError_t launch_attn_merge_wide(const AttnTcArgs& a, int d, cudaStream_t st, bool pdl = false);
 MergeArgs merge_args(const AttnTcArgs& a, int d);
 
 // Message for statekv_last_error(NULL) (errors of calls without a handle).

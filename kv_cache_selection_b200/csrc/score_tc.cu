@@ -14,10 +14,12 @@
 // Each epilogue thread owns one key's TMEM lane, so the column sum of P is a
 // private running sum: no shuffles, no atomics, deterministic.
 //
-// Warp roles (384 threads): warp 0 TMA producer, warp 1 TMEM allocator + MMA
-// issuer, warps 4..11 epilogue: two warpgroups (each covers the 128 TMEM
-// lanes) take alternate chunks, so two chunks are in the epilogue while the
-// MMA fills the next two of the four TMEM accumulators.
+// Warp roles (512 threads): warp 0 TMA producer, warp 1 TMEM allocator + MMA
+// issuer, warps 4..15 epilogue: three warpgroups (each covers the 128 TMEM
+// lanes) take chunks round robin, so up to three chunks are in the epilogue
+// while the MMA fills the fourth of the four TMEM accumulators.  Each
+// epilogue warp reads its lanes 16 columns at a time with the next TMEM load
+// in flight, and frees the accumulator as soon as its last load has landed.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_common.cuh"
@@ -27,12 +29,9 @@ namespace {
 using namespace tc;
 
 constexpr int kStages = 4;
-constexpr int kGroups = 4;                      // epilogue warpgroups (take chunks round robin)
+constexpr int kGroups = 3;                      // epilogue warpgroups (take chunks round robin)
 constexpr int kEpiWarps = 4 * kGroups;
 constexpr int kThreads = 128 + 32 * kEpiWarps;  // warpgroup 0: producer, MMA, two idle warps
-// exponentials of columns with (col & 15) >= kPolyFrom run on the FMA pipe
-// (polynomial), the rest on MUFU; 16 = all on MUFU
-constexpr int kPolyFrom = 16;
 // registers: the launch gives each thread kRegsLaunch; warpgroup 0 drops to
 // kRegsLow and the epilogue warpgroups rise to kRegsHigh within that total
 constexpr int kRegsLaunch = (65536 / kThreads) / 8 * 8 > 168 ? 168 : (65536 / kThreads) / 8 * 8;
@@ -56,6 +55,34 @@ struct Smem {
   static constexpr int kLse = (kAbort + 4 + 15) & ~15;    // [G][n_ic*128] row statistics follow
   static constexpr int kAlloc = kLse + 1024;              // + room to align the base to 1024
 };
+
+// Exponentials of 16 columns (query rows i0 .. i0+15) of one key's TMEM lane,
+// weighted by the rows' negated log2-sum-exps, added to four running sums.
+__device__ __forceinline__ void score_cols16(const uint32_t (&rr)[16], const float* lse2, float scale_log2,
+                                             bool need_mask, bool diag, int i0, int key, int T, float& acc0,
+                                             float& acc1, float& acc2, float& acc3) {
+  const float4* l4 = reinterpret_cast<const float4*>(lse2);
+#pragma unroll
+  for (int j4 = 0; j4 < 4; ++j4) {
+    const float4 lv = l4[j4];  // -lse2 of 4 columns
+    float p0 = ex2_approx(fmaf(__uint_as_float(rr[4 * j4 + 0]), scale_log2, lv.x));
+    float p1 = ex2_approx(fmaf(__uint_as_float(rr[4 * j4 + 1]), scale_log2, lv.y));
+    float p2 = ex2_approx(fmaf(__uint_as_float(rr[4 * j4 + 2]), scale_log2, lv.z));
+    float p3 = ex2_approx(fmaf(__uint_as_float(rr[4 * j4 + 3]), scale_log2, lv.w));
+    if (need_mask) {
+      // frame token `key` is seen by rows i >= key (frame-causal); rows past T do not exist
+      const int i = i0 + 4 * j4;
+      p0 = (i + 0 < T && (!diag || key <= i + 0)) ? p0 : 0.f;
+      p1 = (i + 1 < T && (!diag || key <= i + 1)) ? p1 : 0.f;
+      p2 = (i + 2 < T && (!diag || key <= i + 2)) ? p2 : 0.f;
+      p3 = (i + 3 < T && (!diag || key <= i + 3)) ? p3 : 0.f;
+    }
+    acc0 += p0;
+    acc1 += p1;
+    acc2 += p2;
+    acc3 += p3;
+  }
+}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -229,45 +256,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       // or lie past the frame
       const bool diag = !is_c && a.causal && (i0 < r0 + 127);
       const bool need_mask = diag || i0 + 128 > a.T;
+      // 16 columns at a time; the TMEM load of the next 16 is in flight while
+      // the current 16 are exponentiated, and the accumulator is handed back
+      // to the MMA issuer as soon as its last columns are in registers
+      const uint32_t tb = tmem_addr(tmem, quarter * 32, buf * 128);
+      uint32_t ra[16], rb[16];
+      tmem_ld16(tb, ra);
+      tmem_ld_wait();
 #pragma unroll 1
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t rr[2][32];
-        tmem_ld32(tmem_addr(tmem, quarter * 32, buf * 128 + hf * 64), rr[0]);
-        tmem_ld32(tmem_addr(tmem, quarter * 32, buf * 128 + hf * 64 + 32), rr[1]);
+      for (int q = 0; q < 8; q += 2) {
+        tmem_ld16(tb + 16 * (q + 1), rb);
+        score_cols16(ra, lse2 + 16 * q, a.scale_log2, need_mask, diag, i0 + 16 * q, key, a.T, acc0, acc1, acc2,
+                     acc3);
         tmem_ld_wait();
-#pragma unroll
-        for (int qq = 0; qq < 2; ++qq) {
-          const int q = hf * 2 + qq;
-          const float4* l4 = reinterpret_cast<const float4*>(lse2 + q * 32);
-#pragma unroll
-          for (int j4 = 0; j4 < 8; ++j4) {
-            const float4 lv = l4[j4];  // -lse2 of 4 columns
-            const float x0 = fmaf(__uint_as_float(rr[qq][4 * j4 + 0]), a.scale_log2, lv.x);
-            float p0 = (((4 * j4 + 0) & 15) >= kPolyFrom) ? exp2_poly<4>(x0) : ex2_approx(x0);
-            const float x1 = fmaf(__uint_as_float(rr[qq][4 * j4 + 1]), a.scale_log2, lv.y);
-            float p1 = (((4 * j4 + 1) & 15) >= kPolyFrom) ? exp2_poly<4>(x1) : ex2_approx(x1);
-            const float x2 = fmaf(__uint_as_float(rr[qq][4 * j4 + 2]), a.scale_log2, lv.z);
-            float p2 = (((4 * j4 + 2) & 15) >= kPolyFrom) ? exp2_poly<4>(x2) : ex2_approx(x2);
-            const float x3 = fmaf(__uint_as_float(rr[qq][4 * j4 + 3]), a.scale_log2, lv.w);
-            float p3 = (((4 * j4 + 3) & 15) >= kPolyFrom) ? exp2_poly<4>(x3) : ex2_approx(x3);
-            if (need_mask) {
-              // frame token `key` is seen by rows i >= key (frame-causal); rows past T do not exist
-              const int i = i0 + q * 32 + 4 * j4;
-              p0 = (i + 0 < a.T && (!diag || key <= i + 0)) ? p0 : 0.f;
-              p1 = (i + 1 < a.T && (!diag || key <= i + 1)) ? p1 : 0.f;
-              p2 = (i + 2 < a.T && (!diag || key <= i + 2)) ? p2 : 0.f;
-              p3 = (i + 3 < a.T && (!diag || key <= i + 3)) ? p3 : 0.f;
-            }
-            acc0 += p0;
-            acc1 += p1;
-            acc2 += p2;
-            acc3 += p3;
-          }
+        if (q + 2 < 8) tmem_ld16(tb + 16 * (q + 2), ra);
+        if (q + 2 == 8) {
+          fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_accempty(buf));
         }
+        score_cols16(rb, lse2 + 16 * (q + 1), a.scale_log2, need_mask, diag, i0 + 16 * (q + 1), key, a.T, acc0,
+                     acc1, acc2, acc3);
+        if (q + 2 < 8) tmem_ld_wait();
       }
-      fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_accempty(buf));
     }
     // combine the groups' partial sums of each key row (fixed order)
     float tot = (acc0 + acc1) + (acc2 + acc3);

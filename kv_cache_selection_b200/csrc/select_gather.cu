@@ -53,47 +53,48 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* w
   return r;
 }
 
-// One block per (selection group, stream).  Dynamic shared memory holds the
-// pool's scores (L floats).  Radix select on 8-bit digits, most significant
-// first; each pass is a histogram (warp-aggregated shared atomics) and a
-// suffix count over the 256 bins done with warp shuffles.
-// Appends frame token vectors to D: one 16-byte vector per thread.
-__device__ __forceinline__ void append_vec(const SelectArgs& a, int v) {
-  const int vpr = a.row_bytes / 16;
-  const int per_row = 2 * vpr;  // K and V
-  const int rr = v / per_row;   // (s, t, g) row of the frame
-  if (rr >= a.S * a.T * a.Hkv) return;
-  int e = v - rr * per_row;
-  const bool isv = e >= vpr;
-  if (isv) e -= vpr;
-  const int g = rr % a.Hkv;
-  const int st = rr / a.Hkv;  // s * T + t
-  const int t = st % a.T, s = st / a.T;
-  const long long src = (long long)rr * a.row_bytes;
-  const long long dst = (((long long)s * a.Hkv + g) * a.max_tok + a.d_len + t) * a.row_bytes;
-  const int4 x = __ldg(reinterpret_cast<const int4*>(static_cast<const char*>(isv ? a.vf : a.kf) + src) + e);
-  reinterpret_cast<int4*>(static_cast<char*>(isv ? a.vd : a.kd) + dst)[e] = x;
-  if (g == 0 && !isv && e == 0) a.pos_d[(long long)s * a.max_tok + a.d_len + t] = __ldg(a.pos_f + st);
-}
+// ---------------------------------------------------------------- select
+//
+// One block per (stream, selection group).  The pool's scores are staged in
+// shared memory as their float32 bit patterns (scores are sums of
+// exponentials, >= +0, so the bit patterns order like the values; in recency
+// mode the non-negative positions take their place).  The threshold tau (the
+// B-th largest value) is found by histogram refinement: the values still in
+// play span [umin, umax]; a 4096-bin histogram over that span (bin width
+// 2^shift) locates the bin holding the B-th largest; the bin becomes the new
+// span.  As soon as that bin is one value wide (tau found) or holds at most
+// kBrute candidates, the refinement stops and those candidates are ranked
+// exactly by (value desc, pool index asc).  The result is (tau, need_eq): keep
+// every candidate above tau and the first need_eq candidates equal to tau in
+// pool order, which is position order, so ties go to the lower position.
+constexpr int kBins = 4096;
+constexpr int kBrute = 256;
+
+struct SelShared {
+  alignas(16) uint32_t hist[kBins];
+  uint32_t warp_a[kSelWarps];
+  uint32_t warp_b[kSelWarps];
+  uint32_t list_j[kBrute];
+  uint32_t list_u[kBrute];
+  uint32_t list_n;
+  uint32_t sel_bin, sel_above;
+  uint32_t tau, need_eq;
+};
+
+__device__ __forceinline__ uint32_t warp_min_u32(uint32_t v) { return __reduce_min_sync(0xffffffffu, v); }
+__device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) { return __reduce_max_sync(0xffffffffu, v); }
+__device__ __forceinline__ uint32_t warp_add_u32(uint32_t v) { return __reduce_add_sync(0xffffffffu, v); }
 
 __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) {
-  extern __shared__ float sc[];
-  __shared__ uint32_t hist[257];
-  __shared__ uint32_t bin_tot[8];
-  __shared__ uint32_t warp_tot[32];
-  __shared__ uint32_t sel_bin, sel_above;
+  extern __shared__ uint32_t su[];  // [L] value bits
+  __shared__ SelShared sh;
   pdl_wait();
   pdl_trigger();
   if ((int)blockIdx.x >= a.n_sel_blocks) {
-    // extra blocks: D append, then the merge of key-split partials
-    const int b = blockIdx.x - a.n_sel_blocks;
-    if (b < a.n_app_blocks) {
-      append_vec(a, b * kSelThreads + threadIdx.x);
-    } else {
-      const int t = (b - a.n_app_blocks) * kSelThreads + threadIdx.x;
-      if (a.mrg.d == 128) merge_chunk<128>(a.mrg, t);
-      else merge_chunk<64>(a.mrg, t);
-    }
+    // extra blocks: merge of the attention's key-split partials
+    const int t = (blockIdx.x - a.n_sel_blocks) * kSelThreads + threadIdx.x;
+    if (a.mrg.d == 128) merge_chunk<128>(a.mrg, t);
+    else merge_chunk<64>(a.mrg, t);
     return;
   }
   const int n_groups = a.global ? 1 : a.Hkv;
@@ -103,162 +104,217 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
   const int G0 = a.global ? 0 : grp;
   const int G1 = a.global ? a.Hkv : grp + 1;
 
-  // 1. scores of the pool (global mode sums the KV groups in a fixed order)
-  //    and the pool positions, staged in shared memory; every load of a
-  //    candidate is independent of the others
-  int* posp = reinterpret_cast<int*>(sc + L);
+  // 1. scores of the pool: the KV groups' partial sums added in a fixed order
+  //    (ascending group), written out as the pool scores and staged as bits
   const float* __restrict__ part = a.part + s * a.part_s;
-  const int* __restrict__ pos_c = a.pos_c + ((long long)s * a.Hkv + G0) * a.B;
-  const int* __restrict__ pos_f = a.pos_f + (long long)s * a.T;
+  float* pool_score = a.pool_score + s * a.part_s + (long long)G0 * a.part_g;
   if ((a.part_g & 3) == 0 && (reinterpret_cast<uintptr_t>(part) & 15) == 0) {
-    // four consecutive candidates per thread and group as one 16-byte load,
-    // groups summed in the same fixed order
+    // four consecutive candidates per thread and group as one 16-byte load
     const int n4 = (L + 3) / 4;
     for (int c = threadIdx.x; c < n4; c += kSelThreads) {
       const int j0 = 4 * c;
       const bool full = j0 + 3 < L;
-      int pp[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int j = j0 + e;
-        pp[e] = j < L ? (j < a.m ? __ldg(pos_c + j) : __ldg(pos_f + (j - a.m))) : 0;
-      }
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      // groups in ascending order, eight loads in flight per chunk
       for (int gb = G0; gb < G1; gb += 8) {
+        float4 x[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (gb + u < G1) {
-          const float* src = part + (long long)(gb + u) * a.part_g + j0;
-          float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (full) {
-            x = __ldg(reinterpret_cast<const float4*>(src));
-          } else {
-            x.x = __ldg(src);
-            if (j0 + 1 < L) x.y = __ldg(src + 1);
-            if (j0 + 2 < L) x.z = __ldg(src + 2);
+        for (int u = 0; u < 8; ++u) {
+          x[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (gb + u < G1) {
+            const float* src = part + (long long)(gb + u) * a.part_g + j0;
+            if (full) {
+              x[u] = __ldg(reinterpret_cast<const float4*>(src));
+            } else {
+              x[u].x = __ldg(src);
+              if (j0 + 1 < L) x[u].y = __ldg(src + 1);
+              if (j0 + 2 < L) x[u].z = __ldg(src + 2);
+            }
           }
-          v.x += x.x;
-          v.y += x.y;
-          v.z += x.z;
-          v.w += x.w;
         }
-      }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          v.x += x[u].x;
+          v.y += x[u].y;
+          v.z += x[u].z;
+          v.w += x[u].w;
+        }
       }
       const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         if (j0 + e < L) {
-          sc[j0 + e] = vv[e];
-          posp[j0 + e] = pp[e];
+          pool_score[j0 + e] = vv[e];
+          su[j0 + e] = score_bits(vv[e]);
         }
       }
     }
   } else {
-    constexpr int kBatch = 4;  // candidates per thread whose loads are in flight together
-    for (int jb = 0; jb < L; jb += kBatch * kSelThreads) {
-      float acc[kBatch] = {};
-      int pp[kBatch];
-#pragma unroll
-      for (int q = 0; q < kBatch; ++q) {
-        const int j = jb + q * kSelThreads + threadIdx.x;
-        pp[q] = j < L ? (j < a.m ? __ldg(pos_c + j) : __ldg(pos_f + (j - a.m))) : 0;
-      }
-      // groups in ascending order, eight per chunk with their loads in flight
-      for (int gb = G0; gb < G1; gb += 8) {
-        float pv[kBatch][8];
-#pragma unroll
-        for (int q = 0; q < kBatch; ++q) {
-          const int j = jb + q * kSelThreads + threadIdx.x;
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            pv[q][u] = (j < L && gb + u < G1) ? __ldg(part + (long long)(gb + u) * a.part_g + j) : 0.f;
-        }
-#pragma unroll
-        for (int q = 0; q < kBatch; ++q)
-#pragma unroll
-          for (int u = 0; u < 8; ++u) acc[q] += pv[q][u];
-      }
-#pragma unroll
-      for (int q = 0; q < kBatch; ++q) {
-        const int j = jb + q * kSelThreads + threadIdx.x;
-        if (j < L) {
-          sc[j] = acc[q];
-          posp[j] = pp[q];
-        }
-      }
+    for (int j = threadIdx.x; j < L; j += kSelThreads) {
+      float v = 0.f;
+      for (int g = G0; g < G1; ++g) v += __ldg(part + (long long)g * a.part_g + j);
+      pool_score[j] = v;
+      su[j] = score_bits(v);
     }
   }
-  for (int b = threadIdx.x; b < 257; b += kSelThreads) hist[b] = 0;
-  __syncthreads();
-  for (int j = threadIdx.x; j < L; j += kSelThreads) {
-    a.pool_score[s * a.part_s + (long long)G0 * a.part_g + j] = sc[j];
+  if (a.recency) {
     // recency retention ranks by position: the bit pattern of a non-negative
     // int32 orders like its value, and positions are distinct (no ties)
-    if (a.recency) sc[j] = __int_as_float(max(posp[j], 0));
+    const int* __restrict__ pos_c = a.pos_c + ((long long)s * a.Hkv + G0) * a.B;
+    const int* __restrict__ pos_f = a.pos_f + (long long)s * a.T;
+    for (int j = threadIdx.x; j < L; j += kSelThreads)
+      su[j] = (uint32_t)max(j < a.m ? __ldg(pos_c + j) : __ldg(pos_f + (j - a.m)), 0);
   }
-  if (a.recency) __syncthreads();
+  __syncthreads();
   if (a.B <= 0) return;  // nothing is kept (block-uniform)
 
-  // 2. threshold: the B-th largest score
-  uint32_t tau = 0;
-  int need_eq = 0;  // how many candidates equal to tau are kept
+  // 2. threshold
   const bool keep_all = L <= a.B;
+  uint32_t tau = 0, need_eq = 0;
   if (!keep_all) {
-    uint32_t prefix = 0, pmask = 0;
-    int k = a.B;
-    const int n_iter = (L + kSelThreads - 1) / kSelThreads;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int it = 0; it < n_iter; ++it) {
-        const int j = it * kSelThreads + threadIdx.x;
-        // only candidates that still match the prefix are counted; warps with
-        // none (most of them after the first passes) skip the match entirely
-        bool match = false;
-        uint32_t digit = 0;
+    uint32_t lo = 0, hi = 0xffffffffu;  // span of the values still in play (inclusive)
+    uint32_t need = (uint32_t)a.B;      // how many of them are kept
+    for (int level = 0;; ++level) {
+      // exact span of the values in play
+      uint32_t vmin = 0xffffffffu, vmax = 0u;
+      for (int j = threadIdx.x; j < L; j += kSelThreads) {
+        const uint32_t u = su[j];
+        if (u >= lo && u <= hi) {
+          vmin = min(vmin, u);
+          vmax = max(vmax, u);
+        }
+      }
+      for (int b = threadIdx.x; b < kBins; b += kSelThreads) sh.hist[b] = 0u;
+      vmin = warp_min_u32(vmin);
+      vmax = warp_max_u32(vmax);
+      if (lane == 0) {
+        sh.warp_a[warp] = vmin;
+        sh.warp_b[warp] = vmax;
+      }
+      __syncthreads();
+      vmin = 0xffffffffu;
+      vmax = 0u;
+#pragma unroll 8
+      for (int w = 0; w < kSelWarps; ++w) {
+        vmin = min(vmin, sh.warp_a[w]);
+        vmax = max(vmax, sh.warp_b[w]);
+      }
+      if (vmin == vmax) {  // every value in play is equal: it is tau
+        tau = vmin;
+        need_eq = need;
+        break;
+      }
+      const uint32_t span = vmax - vmin;
+      const int shift = max(0, 32 - __clz(span) - 12);  // (span >> shift) < kBins
+      // histogram of the values in play (warp-aggregated shared atomics)
+      for (int j0 = 0; j0 < L; j0 += kSelThreads) {
+        const int j = j0 + threadIdx.x;
+        bool in = false;
+        uint32_t bin = 0;
         if (j < L) {
-          const uint32_t u = score_bits(sc[j]);
-          match = (u & pmask) == prefix;
-          digit = (u >> shift) & 255u;
+          const uint32_t u = su[j];
+          in = u >= vmin && u <= vmax;
+          bin = (u - vmin) >> shift;
         }
-        const uint32_t act = __ballot_sync(0xffffffffu, match);
-        if (match) {
-          const uint32_t peers = __match_any_sync(act, digit);
-          if (lane == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
+        const uint32_t act = __ballot_sync(0xffffffffu, in);
+        if (in) {
+          const uint32_t peers = __match_any_sync(act, bin);
+          if (lane == __ffs(peers) - 1) atomicAdd(&sh.hist[bin], __popc(peers));
         }
       }
       __syncthreads();
-      // suffix counts: warp w < 8 owns bins [32w, 32w+32)
-      uint32_t suf = 0;
-      if (warp < 8) {
-        suf = hist[warp * 32 + lane];
+      // thread t owns bins [4t, 4t + 4); count of values in bins >= b is the
+      // total minus the exclusive prefix; the bin where it first reaches
+      // `need` from the top holds the need-th largest
+      const uint4 h4 = reinterpret_cast<const uint4*>(sh.hist)[threadIdx.x];
+      const uint32_t mine = h4.x + h4.y + h4.z + h4.w;
+      uint32_t incl = mine;
 #pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          uint32_t n = __shfl_down_sync(0xffffffffu, suf, off);
-          if (lane + off < 32) suf += n;
-        }
-        if (lane == 0) bin_tot[warp] = suf;  // all bins of this warp
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t n = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += n;
       }
+      if (lane == 31) sh.warp_a[warp] = incl;
       __syncthreads();
-      if (warp < 8) {
-        uint32_t higher = 0;  // candidates in bins of higher warps
-        for (int w2 = warp + 1; w2 < 8; ++w2) higher += bin_tot[w2];
-        const uint32_t ge = suf + higher;                                   // digit >= bin
-        const uint32_t gt = ge - hist[warp * 32 + lane];                    // digit > bin
-        if (ge >= (uint32_t)k && gt < (uint32_t)k) {
-          sel_bin = warp * 32 + lane;
-          sel_above = gt;
+      uint32_t before = 0, total = 0;
+#pragma unroll 8
+      for (int w = 0; w < kSelWarps; ++w) {
+        const uint32_t x = sh.warp_a[w];
+        before += w < warp ? x : 0u;
+        total += x;
+      }
+      before += incl - mine;  // values in bins below 4t
+      {
+        const uint32_t hh[4] = {h4.x, h4.y, h4.z, h4.w};
+        uint32_t below = before;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t ge = total - below;       // values in bins >= 4t + e
+          const uint32_t gt = ge - hh[e];          // values in bins > 4t + e
+          if (ge >= need && gt < need) {
+            sh.sel_bin = 4 * threadIdx.x + e;
+            sh.sel_above = gt;
+          }
+          below += hh[e];
         }
       }
+      if (threadIdx.x == 0) sh.list_n = 0u;
       __syncthreads();
-      const uint32_t b = sel_bin;
-      k -= (int)sel_above;
-      prefix |= b << shift;
-      pmask |= 255u << shift;
-      for (int bb = threadIdx.x; bb < 257; bb += kSelThreads) hist[bb] = 0;
-      __syncthreads();
+      const uint32_t b = sh.sel_bin;
+      need -= sh.sel_above;
+      lo = vmin + (b << shift);
+      hi = shift == 0 ? lo : (uint32_t)min((unsigned long long)vmax, (unsigned long long)lo + (1ull << shift) - 1ull);
+      if (shift == 0) {  // the bin is one value
+        tau = lo;
+        need_eq = need;
+        break;
+      }
+      if (sh.hist[b] <= (uint32_t)kBrute) {
+        // rank the bin's candidates exactly: order (value desc, pool index asc)
+        for (int j = threadIdx.x; j < L; j += kSelThreads) {
+          const uint32_t u = su[j];
+          if (u >= lo && u <= hi) {
+            const uint32_t slot = atomicAdd(&sh.list_n, 1u);
+            sh.list_j[slot] = (uint32_t)j;
+            sh.list_u[slot] = u;
+          }
+        }
+        __syncthreads();
+        const uint32_t n = sh.list_n;
+        if (threadIdx.x < n) {
+          const uint32_t uj = sh.list_u[threadIdx.x], jj = sh.list_j[threadIdx.x];
+          uint32_t rank = 0;
+          for (uint32_t k = 0; k < n; ++k) {
+            const uint32_t uk = sh.list_u[k];
+            rank += (uk > uj || (uk == uj && sh.list_j[k] < jj)) ? 1u : 0u;
+          }
+          // the need-th of the bin in that order is tau; the kept ties are the
+          // candidates equal to it ranked before it, plus itself
+          if (rank == need - 1) sh.tau = uj;
+        }
+        __syncthreads();
+        tau = sh.tau;
+        uint32_t eq = 0;
+        if (threadIdx.x < n) {
+          const uint32_t uj = sh.list_u[threadIdx.x], jj = sh.list_j[threadIdx.x];
+          if (uj == tau) {
+            uint32_t rank = 0;
+            for (uint32_t k = 0; k < n; ++k) {
+              const uint32_t uk = sh.list_u[k];
+              rank += (uk > uj || (uk == uj && sh.list_j[k] < jj)) ? 1u : 0u;
+            }
+            eq = rank < need ? 1u : 0u;
+          }
+        }
+        eq = warp_add_u32(eq);
+        if (lane == 0) sh.warp_a[warp] = eq;
+        __syncthreads();
+        need_eq = 0;
+#pragma unroll 8
+        for (int w = 0; w < kSelWarps; ++w) need_eq += sh.warp_a[w];
+        break;
+      }
+      __syncthreads();  // the hist and sel_* reads above finish before the next level rewrites them
     }
-    tau = prefix;
-    need_eq = k;
   }
 
   // 3. compaction in pool (= position) order with one block-wide scan: thread
@@ -272,21 +328,22 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
     if (keep_all) {
       ++n_gt;
     } else {
-      const uint32_t u = score_bits(sc[j]);
+      const uint32_t u = su[j];
       n_gt += u > tau;
       n_eq += u == tau;
     }
   }
-  const uint32_t packed = block_exclusive_scan(n_gt | (n_eq << 16), warp_tot);
-  int eq_seen = (int)(packed >> 16);                               // tied candidates before j_lo
-  int dst = (int)(packed & 0xffffu) + min(eq_seen, need_eq);       // kept candidates before j_lo
+  __syncthreads();  // warp_a is reused by the scan
+  const uint32_t packed = block_exclusive_scan(n_gt | (n_eq << 16), sh.warp_a);
+  uint32_t eq_seen = packed >> 16;                                      // tied candidates before j_lo
+  int dst = (int)(packed & 0xffffu) + (int)min(eq_seen, need_eq);       // kept candidates before j_lo
   int32_t* idx = a.idx + ((long long)s * a.Hkv + G0) * a.B;
   for (int j = j_lo; j < j_hi; ++j) {
     bool keep;
     if (keep_all) {
       keep = true;
     } else {
-      const uint32_t u = score_bits(sc[j]);
+      const uint32_t u = su[j];
       keep = u > tau;
       if (u == tau) keep = eq_seen++ < need_eq;
     }
@@ -297,68 +354,91 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
   }
 }
 
-// One 16-byte vector per thread and step of the grid-stride loop, two steps
-// unrolled so that two kept-index loads and then two row loads are in flight
-// before any store.  Output row r of (stream, KV head): r < m_new gathers C_n
-// from the pool, r >= m_new appends frame token r - m_new to D.  A row pair (K
-// and V) is 2 * row_bytes / 16 vectors.
-__device__ __forceinline__ bool gather_vec(const GatherArgs& a, int v, int per_row, int vpr, int rows,
-                                           const int4** src, int4** dst) {
-  const int rr = v / per_row;
-  int e = v - rr * per_row;
-  const bool isv = e >= vpr;
-  if (isv) e -= vpr;
-  const int row = rr % rows;
-  const int sg = rr / rows;  // s * Hkv + g
-  const int g = sg % a.Hkv;
-  const int s = sg / a.Hkv;
-  const char* sbase;
-  char* dbase;
-  if (row < a.m_new) {
-    const int gsel = a.global ? 0 : g;
-    const int j = __ldg(a.idx + ((long long)s * a.Hkv + gsel) * a.B + row);
-    if (j < 0 || j >= a.m + a.T) return false;  // never taken for a well-formed kept list
-    if (!isv && e == 0) {  // the row's position and score, once per (stream, KV head, slot)
-      a.pos_new[(long long)sg * a.B + row] =
-          j < a.m ? __ldg(a.pos_c + (long long)sg * a.B + j) : __ldg(a.pos_f + (long long)s * a.T + (j - a.m));
-      a.score_new[(long long)sg * a.B + row] = __ldg(a.pool_score + ((long long)s * a.Hkv + gsel) * a.pool_g + j);
-    }
-    if (j < a.m) {
-      sbase = static_cast<const char*>(isv ? a.vc : a.kc) + ((long long)sg * a.B + j) * a.row_bytes;
-    } else {
-      sbase = static_cast<const char*>(isv ? a.vf : a.kf) +
-              (((long long)s * a.T + (j - a.m)) * a.Hkv + g) * a.row_bytes;
-    }
-    dbase = static_cast<char*>(isv ? a.vc_new : a.kc_new) + ((long long)sg * a.B + row) * a.row_bytes;
-  } else {
-    return false;  // rows past m_new do not exist
-  }
-  *src = reinterpret_cast<const int4*>(sbase) + e;
-  *dst = reinterpret_cast<int4*>(dbase) + e;
-  return true;
-}
+// ---------------------------------------------------------------- gather
+//
+// Warp tasks of R rows: a task copies R output rows of one (stream, KV head)
+// -- K and V, VPR 16-byte vectors per row each -- so every lane moves four
+// vectors, all four loads issued before any store.  Tasks [0, n_c) build C_n:
+// the rows' kept pool indices are loaded once per task by R lanes and
+// broadcast; tasks [n_c, n_c + n_d) append R frame tokens of one KV head to D.
+template <int VPR>
+struct GatherShape {
+  static constexpr int kR = 64 / VPR;  // rows per task (four vectors per lane)
+  static constexpr int kU = 4;
+};
 
-__global__ void __launch_bounds__(256) gather_append_kernel(GatherArgs a) {
+template <int VPR>
+__global__ void __launch_bounds__(256) gather_append_kernel(GatherArgs a, int n_c_tasks, int n_tasks) {
+  constexpr int R = GatherShape<VPR>::kR, U = GatherShape<VPR>::kU;
   pdl_wait();
   pdl_trigger();
-  const int vpr = a.row_bytes / 16;
-  const int per_row = 2 * vpr;
-  const int rows = a.m_new;
-  const int total = a.S * a.Hkv * rows * per_row;
-  const int stride = gridDim.x * blockDim.x;
-  for (int v0 = blockIdx.x * blockDim.x + threadIdx.x; v0 < total; v0 += 2 * stride) {
-    const int v1 = v0 + stride;
-    const int4* s0 = nullptr;
-    const int4* s1 = nullptr;
-    int4* d0 = nullptr;
-    int4* d1 = nullptr;
-    const bool ok0 = gather_vec(a, v0, per_row, vpr, rows, &s0, &d0);
-    const bool ok1 = v1 < total && gather_vec(a, v1, per_row, vpr, rows, &s1, &d1);
-    int4 x0, x1;
-    if (ok0) x0 = __ldg(s0);
-    if (ok1) x1 = __ldg(s1);
-    if (ok0) *d0 = x0;
-    if (ok1) *d1 = x1;
+  const int lane = threadIdx.x & 31;
+  const int warps_total = gridDim.x * (blockDim.x >> 5);
+  const int c_blocks = (a.m_new + R - 1) / R;   // C tasks per (stream, KV head)
+  const int d_blocks = (a.T + R - 1) / R;       // D tasks per (stream, KV head)
+  for (int task = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); task < n_tasks; task += warps_total) {
+    const bool is_c = task < n_c_tasks;
+    const int t2 = is_c ? task : task - n_c_tasks;
+    const int per = is_c ? c_blocks : d_blocks;
+    const int sg = t2 / per;                     // s * Hkv + g
+    const int r0 = (t2 - sg * per) * R;
+    const int g = sg % a.Hkv, s = sg / a.Hkv;
+    const int n_rows = min(R, (is_c ? a.m_new : a.T) - r0);
+    const int4* src[U];
+    int4* dst[U];
+    bool ok[U];
+    if (is_c) {
+      const int gsel = a.global ? 0 : g;
+      int j = -1;
+      if (lane < n_rows) {
+        j = __ldg(a.idx + ((long long)s * a.Hkv + gsel) * a.B + r0 + lane);
+        if (j < 0 || j >= a.m + a.T) j = -1;  // never taken for a well-formed kept list
+        if (j >= 0) {
+          a.pos_new[(long long)sg * a.B + r0 + lane] =
+              j < a.m ? __ldg(a.pos_c + (long long)sg * a.B + j) : __ldg(a.pos_f + (long long)s * a.T + (j - a.m));
+          a.score_new[(long long)sg * a.B + r0 + lane] =
+              __ldg(a.pool_score + ((long long)s * a.Hkv + gsel) * a.pool_g + j);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int e = lane + 32 * u;
+        const int rl = e / (2 * VPR), w = e % (2 * VPR);
+        const bool isv = w >= VPR;
+        const int col = isv ? w - VPR : w;
+        const int jr = __shfl_sync(0xffffffffu, j, rl);
+        ok[u] = rl < n_rows && jr >= 0;
+        const char* sb;
+        if (jr < a.m) sb = static_cast<const char*>(isv ? a.vc : a.kc) + ((long long)sg * a.B + jr) * a.row_bytes;
+        else sb = static_cast<const char*>(isv ? a.vf : a.kf) + (((long long)s * a.T + (jr - a.m)) * a.Hkv + g) * a.row_bytes;
+        src[u] = reinterpret_cast<const int4*>(sb) + col;
+        dst[u] = reinterpret_cast<int4*>(static_cast<char*>(isv ? a.vc_new : a.kc_new) +
+                                         ((long long)sg * a.B + r0 + rl) * a.row_bytes) + col;
+      }
+    } else {
+      if (g == 0 && lane < n_rows)
+        a.pos_d[(long long)s * a.max_tok + a.d_len + r0 + lane] = __ldg(a.pos_f + (long long)s * a.T + r0 + lane);
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int e = lane + 32 * u;
+        const int rl = e / (2 * VPR), w = e % (2 * VPR);
+        const bool isv = w >= VPR;
+        const int col = isv ? w - VPR : w;
+        const int t = r0 + rl;
+        ok[u] = rl < n_rows;
+        src[u] = reinterpret_cast<const int4*>(static_cast<const char*>(isv ? a.vf : a.kf) +
+                                               (((long long)s * a.T + t) * a.Hkv + g) * a.row_bytes) + col;
+        dst[u] = reinterpret_cast<int4*>(static_cast<char*>(isv ? a.vd : a.kd) +
+                                         (((long long)s * a.Hkv + g) * a.max_tok + a.d_len + t) * a.row_bytes) + col;
+      }
+    }
+    int4 x[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (ok[u]) x[u] = __ldg(src[u]);
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (ok[u]) *dst[u] = x[u];
   }
 }
 
@@ -369,34 +449,45 @@ cudaError_t launch_select(const SelectArgs& a_in, int S, cudaStream_t st, bool p
   const int L = a.m + a.T;
   const int n_groups = a.global ? 1 : a.Hkv;
   a.n_sel_blocks = n_groups * S;
-  const long long app_vecs = (long long)S * a.T * a.Hkv * 2 * (a.row_bytes / 16);
-  a.n_app_blocks = (int)((app_vecs + kSelThreads - 1) / kSelThreads);
-  a.S = S;
   if (a.mrg.n_split > 1) {
     const long long mrg_threads = (long long)a.mrg.S * a.mrg.Hq * a.mrg.T * (a.mrg.d / 8);
     a.n_mrg_blocks = (int)((mrg_threads + kSelThreads - 1) / kSelThreads);
   } else {
     a.n_mrg_blocks = 0;
   }
-  const size_t smem = (size_t)L * (sizeof(float) + sizeof(int));
+  const size_t smem = (size_t)L * sizeof(uint32_t);
   // the default 48 KB per block covers static and dynamic shared memory
-  // together; the kernel's static arrays take ~1.2 KB, so opt in well before
-  if (smem > 40 * 1024) {
+  // together; the kernel's static arrays take ~19 KB, so opt in above 24 KB
+  if (smem > 24 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(select_topb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
   }
-  return launch_kernel(select_topb_kernel, dim3(a.n_sel_blocks + a.n_app_blocks + a.n_mrg_blocks),
-                       dim3(kSelThreads), smem, st, pdl, a);
+  return launch_kernel(select_topb_kernel, dim3(a.n_sel_blocks + a.n_mrg_blocks), dim3(kSelThreads), smem, st,
+                       pdl, a);
+}
+
+template <int VPR>
+static cudaError_t launch_gather_vpr(const GatherArgs& a, int n_sm, cudaStream_t st, bool pdl) {
+  constexpr int R = GatherShape<VPR>::kR;
+  const int per_c = (a.m_new + R - 1) / R, per_d = (a.T + R - 1) / R;
+  const long long n_c = (long long)a.S * a.Hkv * per_c;
+  const long long n_tasks = n_c + (long long)a.S * a.Hkv * per_d;
+  if (n_tasks == 0) return cudaSuccess;
+  long long blocks = (n_tasks + 7) / 8;        // eight warps per block
+  const long long cap = (long long)n_sm * 8;   // one resident wave
+  if (blocks > cap) blocks = cap;
+  return launch_kernel(gather_append_kernel<VPR>, dim3((unsigned)blocks), dim3(256), 0, st, pdl, a, (int)n_c,
+                       (int)n_tasks);
 }
 
 cudaError_t launch_gather(const GatherArgs& a, int n_sm, cudaStream_t st, bool pdl) {
-  const long long vecs = (long long)a.S * a.Hkv * a.m_new * 2 * (a.row_bytes / 16);
-  if (vecs == 0) return cudaSuccess;
-  long long blocks = (vecs + 2 * 256 - 1) / (2 * 256);  // two vectors per thread
-  const long long cap = (long long)n_sm * 8;           // one resident wave at 8 blocks per SM
-  if (blocks > cap) blocks = cap;
-  return launch_kernel(gather_append_kernel, dim3((unsigned)blocks), dim3(256), 0, st, pdl, a);
+  switch (a.row_bytes / 16) {
+    case 8: return launch_gather_vpr<8>(a, n_sm, st, pdl);
+    case 16: return launch_gather_vpr<16>(a, n_sm, st, pdl);
+    case 32: return launch_gather_vpr<32>(a, n_sm, st, pdl);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace skv

@@ -58,13 +58,23 @@ struct statekv_handle {
   __nv_bfloat16* o_part = nullptr;  // attention key-split partials (bf16 path)
   float* ml_part = nullptr;
   int max_split = 1;
-  // staging for statekv_prefill_frame_host (allocated on first use)
-  void* stage_q = nullptr;
-  void* stage_k = nullptr;
-  void* stage_v = nullptr;
-  void* stage_out = nullptr;
-  int32_t* stage_pos = nullptr;
+  // statekv_prefill_frame_host: two staging sets used in turn, a copy stream
+  // for the host-to-device copies, and the events that order them (created on
+  // first use)
+  void* stage_q[2] = {nullptr, nullptr};
+  void* stage_k[2] = {nullptr, nullptr};
+  void* stage_v[2] = {nullptr, nullptr};
+  void* stage_out[2] = {nullptr, nullptr};
+  int32_t* stage_pos[2] = {nullptr, nullptr};
+  int stage_next = 0;
+  cudaStream_t copy_stream = nullptr;
+  cudaEvent_t ev_h2d[2] = {nullptr, nullptr};   // inputs of set b are on the device
+  cudaEvent_t ev_stage_free[2] = {nullptr, nullptr};  // the step and copy-out of set b are done
   int last_pool_len = 0;
+  // key-split partials of statekv_decode (float32), grown on demand
+  float* dec_o = nullptr;
+  float* dec_ml = nullptr;
+  size_t dec_o_bytes = 0, dec_ml_bytes = 0;
   std::string err;
   std::vector<void*> allocs;
   // launch accounting and optional per-stage event timing
@@ -272,6 +282,8 @@ int full_causal_tc(const void* q, const void* k, const void* v, int n_seq, int N
   ta.n_split = skv::attn_tc_splits(n_seq, Hq, Hkv, N, 0, n_sm);
   ta.nC = 0;
   ta.nF = ta.n_it;
+  ta.stack = 0;
+  ta.q_rows = 128;
   ta.scale_log2 = skv::kLog2e / sqrtf((float)d);
   {
     std::lock_guard<std::mutex> lk(g_fc_mu);
@@ -462,6 +474,8 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
     ta.n_split = std::min(h->max_split, skv::attn_tc_splits(S, Hq, Hkv, T, m, h->n_sm));
     ta.nC = (m + 127) / 128;
     ta.nF = ta.n_it;
+  ta.stack = 0;
+  ta.q_rows = 128;
     ta.scale_log2 = scale_log2;
     ta.err = h->dev_err;
     {
@@ -471,7 +485,17 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
       sc.done();
     }
     n_split = ta.n_split;
-    if (n_split > 1) mrg = skv::merge_args(ta, d);
+    if (n_split > 1) {
+      if (h->prof) {
+        // timed runs charge the merge of the key splits to the attention stage
+        // by launching it on its own; otherwise it rides in the select launch
+        StageScope sc(h, st, STATEKV_STAGE_ATTENTION_COMBINE);
+        if ((e = skv::launch_attn_combine(ta, d, st, true)) != cudaSuccess) return launch_err(h, e, "attention merge");
+        sc.done();
+      } else {
+        mrg = skv::merge_args(ta, d);
+      }
+    }
   } else {
     StageScope sc(h, st, STATEKV_STAGE_ATTENTION);
     if ((e = skv::launch_attn_simt(aa, h->dtype, d, S, st)) != cudaSuccess) return launch_err(h, e, "attention");
@@ -544,14 +568,6 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
   se.B = B;
   se.global = h->select != STATEKV_SELECT_PER_KV_HEAD;  // recency keeps one set per layer too
   se.recency = h->select == STATEKV_SELECT_RECENCY;
-  se.kf = k;
-  se.vf = v;
-  se.kd = L->kd;
-  se.vd = L->vd;
-  se.pos_d = L->posd;
-  se.row_bytes = (int)(d * h->esize);
-  se.d_len = L->frames * T;
-  se.max_tok = h->max_frames * T;
   se.mrg = mrg;
   {
     StageScope sc(h, st, STATEKV_STAGE_SELECT);
@@ -609,24 +625,171 @@ int statekv_prefill_frame_host(statekv_t h, int layer, const void* q, const void
   const size_t kb = (size_t)h->S * h->T * h->Hkv * h->d * h->esize;
   const size_t pb = (size_t)h->S * h->T * 4;
   int rc;
-  if (!h->stage_q) {
-    if ((rc = dev_alloc(h, &h->stage_q, qb)) || (rc = dev_alloc(h, &h->stage_k, kb)) ||
-        (rc = dev_alloc(h, &h->stage_v, kb)) || (rc = dev_alloc(h, &h->stage_out, qb)) ||
-        (rc = dev_alloc(h, (void**)&h->stage_pos, pb)))
-      return rc;
-  }
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if ((e = cudaMemcpyAsync(h->stage_q, q, qb, cudaMemcpyHostToDevice, st)) != cudaSuccess ||
-      (e = cudaMemcpyAsync(h->stage_k, k, kb, cudaMemcpyHostToDevice, st)) != cudaSuccess ||
-      (e = cudaMemcpyAsync(h->stage_v, v, kb, cudaMemcpyHostToDevice, st)) != cudaSuccess ||
-      (e = cudaMemcpyAsync(h->stage_pos, pos, pb, cudaMemcpyHostToDevice, st)) != cudaSuccess)
+  if (!h->stage_q[0]) {
+    for (int b = 0; b < 2; ++b)
+      if ((rc = dev_alloc(h, &h->stage_q[b], qb)) || (rc = dev_alloc(h, &h->stage_k[b], kb)) ||
+          (rc = dev_alloc(h, &h->stage_v[b], kb)) || (rc = dev_alloc(h, &h->stage_out[b], qb)) ||
+          (rc = dev_alloc(h, (void**)&h->stage_pos[b], pb)))
+        return rc;
+    if ((e = cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking)) != cudaSuccess)
+      return set_err(h, STATEKV_ERR_CUDA, "copy stream: %s", cudaGetErrorString(e));
+    for (int b = 0; b < 2; ++b)
+      if ((e = cudaEventCreateWithFlags(&h->ev_h2d[b], cudaEventDisableTiming)) != cudaSuccess ||
+          (e = cudaEventCreateWithFlags(&h->ev_stage_free[b], cudaEventDisableTiming)) != cudaSuccess)
+        return set_err(h, STATEKV_ERR_CUDA, "staging events: %s", cudaGetErrorString(e));
+  }
+  // the step's own refusals, checked before anything is enqueued
+  if (layer < 0) return set_err(h, STATEKV_ERR_INVALID_ARG, "negative layer %d", layer);
+  if ((size_t)layer < h->layers.size() && h->layers[layer].ready && h->layers[layer].frames >= h->max_frames)
+    return set_err(h, STATEKV_ERR_CAPACITY, "layer %d already holds max_frames=%d frames", layer, h->max_frames);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int b = h->stage_next;
+  // The inputs of this call go to staging set b on the copy stream once the
+  // step that last read set b is done, so they can arrive while the previous
+  // call's step still runs; the step waits for them, then copies out back on
+  // the caller's stream.
+  if ((e = cudaStreamWaitEvent(h->copy_stream, h->ev_stage_free[b], 0)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(h->stage_q[b], q, qb, cudaMemcpyHostToDevice, h->copy_stream)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(h->stage_k[b], k, kb, cudaMemcpyHostToDevice, h->copy_stream)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(h->stage_v[b], v, kb, cudaMemcpyHostToDevice, h->copy_stream)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(h->stage_pos[b], pos, pb, cudaMemcpyHostToDevice, h->copy_stream)) != cudaSuccess ||
+      (e = cudaEventRecord(h->ev_h2d[b], h->copy_stream)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(st, h->ev_h2d[b], 0)) != cudaSuccess)
     return set_err(h, STATEKV_ERR_CUDA, "host-to-device copy failed: %s", cudaGetErrorString(e));
-  rc = statekv_prefill_frame(h, layer, h->stage_q, h->stage_k, h->stage_v, h->stage_pos, h->stage_out,
-                             stream);
+  rc = statekv_prefill_frame(h, layer, h->stage_q[b], h->stage_k[b], h->stage_v[b], h->stage_pos[b],
+                             h->stage_out[b], stream);
   if (rc) return rc;
-  if ((e = cudaMemcpyAsync(out, h->stage_out, qb, cudaMemcpyDeviceToHost, st)) != cudaSuccess)
+  if ((e = cudaMemcpyAsync(out, h->stage_out[b], qb, cudaMemcpyDeviceToHost, st)) != cudaSuccess ||
+      (e = cudaEventRecord(h->ev_stage_free[b], st)) != cudaSuccess)
     return set_err(h, STATEKV_ERR_CUDA, "device-to-host copy failed: %s", cudaGetErrorString(e));
+  h->stage_next = b ^ 1;
+  return STATEKV_OK;
+}
+
+int statekv_decode(statekv_t h, int layer, const void* q, const void* k, const void* v, int n_text, void* out,
+                   float* lse, void* stream) {
+  if (!h) return set_err(nullptr, STATEKV_ERR_INVALID_ARG, "null handle");
+  if (!q || !k || !v || !out) return set_err(h, STATEKV_ERR_INVALID_ARG, "null input/output pointer");
+  if (n_text < 1) return set_err(h, STATEKV_ERR_INVALID_ARG, "n_text=%d must be >= 1", n_text);
+  if (((uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)out) & 15)
+    return set_err(h, STATEKV_ERR_INVALID_ARG, "q/k/v/out must be 16-byte aligned");
+  if (lse && ((uintptr_t)lse & 3)) return set_err(h, STATEKV_ERR_INVALID_ARG, "lse must be 4-byte aligned");
+  if (layer < 0 || (size_t)layer >= h->layers.size() || !h->layers[layer].ready)
+    return set_err(h, STATEKV_ERR_INVALID_ARG, "unknown layer %d", layer);
+  const LayerState& L = h->layers[layer];
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int S = h->S, Hq = h->Hq, Hkv = h->Hkv, d = h->d, T = h->T, G = Hq / Hkv;
+  const int N = L.frames * T;                 // tokens in D
+  const long long max_tok = (long long)h->max_frames * T;
+  const float scale_log2 = skv::kLog2e / sqrtf((float)d);
+  cudaError_t e;
+  if (h->dtype != STATEKV_BF16) {
+    skv::AttnArgs aa{};
+    aa.q = q;
+    aa.q_s = (long long)n_text * Hq * d;
+    aa.q_row = Hq * d;
+    aa.ka = L.kd;
+    aa.va = L.vd;
+    aa.a_s = (long long)Hkv * max_tok * d;
+    aa.a_g = max_tok * d;
+    aa.m = N;
+    aa.kb = k;
+    aa.vb = v;
+    aa.b_s = (long long)n_text * Hkv * d;
+    aa.b_row = Hkv * d;
+    aa.nb = n_text;
+    aa.out = out;
+    aa.lse = lse;
+    aa.lse_s = (long long)Hq * n_text;
+    aa.n_rows = n_text;
+    aa.Hq = Hq;
+    aa.Hkv = Hkv;
+    aa.causal = 1;
+    aa.scale_log2 = scale_log2;
+    StageScope sc(h, st, STATEKV_STAGE_DECODE);
+    if ((e = skv::launch_attn_simt(aa, h->dtype, d, S, st)) != cudaSuccess) return launch_err(h, e, "decode");
+    sc.done();
+    return STATEKV_OK;
+  }
+  // tensor cores: each query tile stacks the G heads of a KV group, so every
+  // D tile is read once per group; key splits fill the SMs
+  skv::AttnTcArgs ta{};
+  const int ri = 128 / G;
+  ta.out = out;
+  ta.out_s = (long long)n_text * Hq * d;
+  ta.out_row = Hq * d;
+  ta.lse = lse;
+  ta.lse_s = (long long)Hq * n_text;
+  ta.m = N;
+  ta.T = n_text;
+  ta.Hq = Hq;
+  ta.Hkv = Hkv;
+  ta.causal = 1;
+  ta.S = S;
+  ta.stack = G;
+  ta.q_rows = G * ri;
+  ta.n_it = (n_text + ri - 1) / ri;
+  ta.n_pairs = (ta.n_it + 1) / 2;
+  ta.nC = (N + 127) / 128;
+  ta.nF = (n_text + 127) / 128;
+  ta.scale_log2 = scale_log2;
+  ta.err = h->dev_err;
+  const int units = S * Hkv * ta.n_pairs;
+  int split = std::max(1, h->n_sm / std::max(units, 1));
+  split = std::min(split, std::min(ta.nC + ta.nF, 256));
+  ta.n_split = split;
+  if (split > 1) {
+    const size_t ob = (size_t)S * Hq * split * n_text * d * 4, mb = (size_t)S * Hq * split * n_text * 4;
+    if (h->dec_o_bytes < ob) {
+      if (h->dec_o) cudaFree(h->dec_o);
+      h->dec_o = nullptr;
+      h->dec_o_bytes = 0;
+      if (cudaMalloc((void**)&h->dec_o, ob) != cudaSuccess) {
+        cudaGetLastError();
+        return set_err(h, STATEKV_ERR_OOM, "decode scratch of %zu bytes", ob);
+      }
+      h->dec_o_bytes = ob;
+    }
+    if (h->dec_ml_bytes < mb) {
+      if (h->dec_ml) cudaFree(h->dec_ml);
+      h->dec_ml = nullptr;
+      h->dec_ml_bytes = 0;
+      if (cudaMalloc((void**)&h->dec_ml, mb) != cudaSuccess) {
+        cudaGetLastError();
+        return set_err(h, STATEKV_ERR_OOM, "decode scratch of %zu bytes", mb);
+      }
+      h->dec_ml_bytes = mb;
+    }
+    ta.o_part32 = h->dec_o;
+    ta.ml_part = h->dec_ml;
+  }
+  const uint64_t D = d;
+  const uint64_t dq[4] = {D, (uint64_t)Hq, (uint64_t)n_text, (uint64_t)S};
+  const uint64_t sq[3] = {D * 2, (uint64_t)Hq * D * 2, (uint64_t)n_text * Hq * D * 2};
+  const uint32_t bq[4] = {64, (uint32_t)G, (uint32_t)ri, 1};
+  const uint64_t dd[4] = {D, (uint64_t)max_tok, (uint64_t)Hkv, (uint64_t)S};
+  const uint64_t sd[3] = {D * 2, (uint64_t)max_tok * D * 2, (uint64_t)Hkv * max_tok * D * 2};
+  const uint32_t bd[4] = {64, 128, 1, 1};
+  const uint64_t dk[4] = {D, (uint64_t)Hkv, (uint64_t)n_text, (uint64_t)S};
+  const uint64_t sk[3] = {D * 2, (uint64_t)Hkv * D * 2, (uint64_t)n_text * Hkv * D * 2};
+  const uint32_t bk[4] = {64, 1, 128, 1};
+  CUtensorMap tq, tkd, tvd, tk, tv;
+  int r;
+  if ((r = skv::encode_tmap_bf16_4d(&tq, q, dq, sq, bq)) || (r = skv::encode_tmap_bf16_4d(&tkd, L.kd, dd, sd, bd)) ||
+      (r = skv::encode_tmap_bf16_4d(&tvd, L.vd, dd, sd, bd)) || (r = skv::encode_tmap_bf16_4d(&tk, k, dk, sk, bk)) ||
+      (r = skv::encode_tmap_bf16_4d(&tv, v, dk, sk, bk)))
+    return set_err(h, STATEKV_ERR_CUDA, "TMA tensor map encoding failed (CUresult %d)", r);
+  {
+    StageScope sc(h, st, STATEKV_STAGE_DECODE);
+    if ((e = skv::launch_attn_tc(tq, tkd, tvd, tk, tv, ta, d, st)) != cudaSuccess) return launch_err(h, e, "decode");
+    sc.done();
+  }
+  if (split > 1) {
+    StageScope sc(h, st, STATEKV_STAGE_DECODE_COMBINE);
+    if ((e = skv::launch_attn_merge_wide(ta, d, st, true)) != cudaSuccess) return launch_err(h, e, "decode merge");
+    sc.done();
+  }
   return STATEKV_OK;
 }
 
@@ -727,8 +890,15 @@ int statekv_destroy(statekv_t h) {
     cudaEventDestroy(r.a);
     cudaEventDestroy(r.b);
   }
+  for (int b = 0; b < 2; ++b) {
+    if (h->ev_h2d[b]) cudaEventDestroy(h->ev_h2d[b]);
+    if (h->ev_stage_free[b]) cudaEventDestroy(h->ev_stage_free[b]);
+  }
+  if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
   for (cudaEvent_t e : h->ev_free) cudaEventDestroy(e);
   for (void* p : h->allocs) cudaFree(p);
+  if (h->dec_o) cudaFree(h->dec_o);
+  if (h->dec_ml) cudaFree(h->dec_ml);
   delete h;
   return STATEKV_OK;
 }

@@ -205,14 +205,6 @@ extern "C" int statekv_step_noalloc(int Hq, int Hkv, int d, int T, int B, int dt
   se.B = B;
   se.global = global;
   se.recency = select_mode == STATEKV_SELECT_RECENCY;
-  se.kf = k;
-  se.vf = v;
-  se.kd = kd;
-  se.vd = vd;
-  se.pos_d = posd;
-  se.row_bytes = d * (dtype == STATEKV_BF16 ? 2 : 4);
-  se.d_len = d_len;
-  se.max_tok = max_tok;
   if ((e = skv::launch_select(se, 1, st)) != cudaSuccess)
     return fail(STATEKV_ERR_CUDA, "select launch: %s", cudaGetErrorString(e));
 

@@ -163,6 +163,19 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Wait for this thread's outstanding TMEM loads, with the destination
+// registers of one load as operands, so that no use of them is scheduled
+// before the wait (the load's results arrive asynchronously).
+__device__ __forceinline__ void tmem_ld_wait_dep(uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+        "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+        "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+        "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+      :
+      : "memory");
+}
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
@@ -290,33 +303,6 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int* er
   uint32_t ok = 1;
   if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, err, code, abort_flag) ? 1u : 0u;
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
-}
-
-// 2^x on the FMA pipe instead of the MUFU unit (for kernels whose
-// exponentials outnumber what MUFU can issue).  Range reduction: j = round(x)
-// by adding 1.5 * 2^23 (the integer lands in the low mantissa bits),
-// f = x - j in [-1/2, 1/2]; 2^f by a polynomial whose coefficients were fitted
-// for minimal relative error on that interval (degree 3: 1.0e-4, degree 4:
-// 2.9e-6, evaluated in float32 Horner form); 2^j is applied by adding j to the
-// exponent field.  x is clamped at -120, so inputs below that give about
-// 2^-120, not 0: callers mask explicitly where exact zeros matter.
-template <int DEG>
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -120.f);
-  const float t = x + 12582912.f;
-  const float j = t - 12582912.f;
-  const float f = x - j;
-  float p;
-  if (DEG == 3) {
-    p = fmaf(f, 0.055008821189403534f, 0.2422107756137848f);
-    p = fmaf(f, p, 0.6932829022407532f);
-  } else {
-    p = fmaf(f, 0.009582837112247944f, 0.05590641498565674f);
-    p = fmaf(f, p, 0.24024099111557007f);
-    p = fmaf(f, p, 0.6931241750717163f);
-  }
-  p = fmaf(f, p, 1.f);
-  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {

@@ -21,7 +21,7 @@ BF16, F32 = 0, 1
 MASKS = {"frame_causal": 0, "frame_bidir": 1}
 SELECTS = {"global": 0, "per_kv_head": 1, "recency": 2}
 N_STAGES = 8
-STAGES = ["attention", "attention_combine", "score", "select", "gather", None, None, None]
+STAGES = ["attention", "attention_combine", "score", "select", "gather", "decode", "decode_combine", None]
 ERRORS = {0: "OK", -1: "INVALID_ARG", -2: "UNSUPPORTED", -3: "CAPACITY", -4: "OOM", -5: "CUDA"}
 
 if not os.path.exists(LIB_PATH):
@@ -53,6 +53,7 @@ _SIGS = {
     "statekv_destroy": (_i, [_vp]),
     "statekv_last_error": (ctypes.c_char_p, [_vp]),
     "statekv_step_noalloc": (_i, [_i] * 8 + [_vp] * 7 + [_i] + [_vp] * 8 + [_i, _i, _vp]),
+    "statekv_decode": (_i, [_vp, _i, _vp, _vp, _vp, _i, _vp, _vp, _vp]),
     "full_causal_prefill": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp]),
     "full_causal_prefill_batched": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp]),
 }
@@ -199,6 +200,27 @@ class StateKV:
                                             pos.data_ptr(), out.data_ptr(), _stream_ptr(stream))
         _check(rc, self._h)
         return out
+
+    def decode(self, layer, q, k, v, out=None, lse=None, with_lse=True, stream=None):
+        """Attention of n text tokens over the layer's detailed state D and
+        causally over themselves: q [.., n, Hq, d], k/v [.., n, Hkv, d].
+        Returns (out, lse [.., Hq, n] or None)."""
+        L = self._lead()
+        n = q.shape[-3]
+        _need(q, L + (n, self.Hq, self.d), self.dtype, "q")
+        _need(k, L + (n, self.Hkv, self.d), self.dtype, "k")
+        _need(v, L + (n, self.Hkv, self.d), self.dtype, "v")
+        if out is None:
+            out = torch.empty_like(q)
+        _need(out, L + (n, self.Hq, self.d), self.dtype, "out")
+        if lse is None and with_lse:
+            lse = torch.empty(L + (self.Hq, n), dtype=torch.float32, device=q.device)
+        if lse is not None:
+            _need(lse, L + (self.Hq, n), torch.float32, "lse")
+        rc = lib.statekv_decode(self._h, layer, q.data_ptr(), k.data_ptr(), v.data_ptr(), n, out.data_ptr(),
+                                lse.data_ptr() if lse is not None else None, _stream_ptr(stream))
+        _check(rc, self._h)
+        return out, lse
 
     def frames(self, layer) -> int:
         return lib.statekv_frames(self._h, layer)

@@ -444,3 +444,85 @@ def test_diagnostics_library_fed_match_oracle_fed():
         assert abs(rg["captured"][name] - ro["captured"][name]) <= 1e-3
     for h in list(sel.values()) + [full]:
         h.close()
+
+
+def _decode_case(wl, n_frames, n_text, dtype, device_frames=False, n_streams=1):
+    """Fill a handle's D with n_frames frames, then decode n_text text tokens
+    over it; compare with the oracle's decode attention on the same D."""
+    S = _skv()
+    dev = torch.device("cuda")
+    h = S.StateKV(wl.Hq, wl.Hkv, wl.d, wl.T, wl.B, max_frames=max(n_frames, 1), dtype=dtype,
+                  n_streams=n_streams)
+    h.reserve_layers(1)
+    if device_frames:
+        per = [Syn.gen_frames_device(wl, n_frames, stream=s, device=dev) for s in range(n_streams)]
+        for n in range(n_frames):
+            args = [torch.stack([p[i][n] for p in per]) if n_streams > 1 else per[0][i][n] for i in range(4)]
+            h.prefill_frame(0, *args)
+        del per
+    else:
+        for n in range(n_frames):
+            fr = [Syn.gen_frame(wl, n, stream=s) for s in range(n_streams)]
+            args = [(torch.stack([f[i] for f in fr]) if n_streams > 1 else fr[0][i]).to(dev) for i in range(4)]
+            h.prefill_frame(0, *args)
+    # text tokens: the recipe's next frame, first n_text tokens
+    wl_txt = Syn.workload(wl.name, T=n_text, dist="iid", n_sinks=0, drift=0)
+    txt = [Syn.gen_frame(wl_txt, n_frames, stream=s) for s in range(n_streams)]
+    q = torch.stack([t[0] for t in txt]) if n_streams > 1 else txt[0][0]
+    k = torch.stack([t[1] for t in txt]) if n_streams > 1 else txt[0][1]
+    v = torch.stack([t[2] for t in txt]) if n_streams > 1 else txt[0][2]
+    out, lse = h.decode(0, q.to(dev), k.to(dev), v.to(dev))
+    torch.cuda.synchronize()
+    D = h.get_detailed(0)
+    N = D["len"]
+    assert N == n_frames * wl.T
+    for s in range(n_streams):
+        DK = D["k"][s, :, :N].cpu()
+        DV = D["v"][s, :, :N].cpu()
+        ref_out, ref_lse = O.decode_attention(DK, DV, *(x[s] if n_streams > 1 else x for x in (q, k, v)))
+        P.check_out(out[s] if n_streams > 1 else out, ref_out, dtype, what=f"decode stream {s}")
+        P.check_lse(lse[s] if n_streams > 1 else lse, ref_lse, dtype)
+    assert h.device_status() == 0
+    h.close()
+
+
+@cuda
+@pytest.mark.parametrize("n_text", [1, 5, 16])
+def test_decode_tiny_f32(n_text):
+    _decode_case(Syn.workload("tiny"), 8, n_text, "f32")
+
+
+@cuda
+@pytest.mark.parametrize("n_text", [1, 7, 18, 19, 37, 130])
+def test_decode_8b_shape(n_text):
+    """8B layer shape after 16 frames (4096 D tokens): one stacked query tile
+    (18 rows of 7 heads), a partly filled pair, two pairs, and text longer than
+    one 128-token key tile."""
+    _decode_case(Syn.workload("8b_layer"), 16, n_text, "bf16")
+
+
+@cuda
+@pytest.mark.parametrize("d,Hq,Hkv", [(64, 14, 2), (128, 8, 8)])
+def test_decode_other_groups(d, Hq, Hkv):
+    """Group sizes 7 and 1 and head dim 64; D that does not fill its last tile."""
+    wl = Syn.workload("1b_layer", Hq=Hq, Hkv=Hkv, d=d, T=100, B=256)
+    _decode_case(wl, 5, 9, "bf16")
+
+
+@cuda
+def test_decode_batched_streams():
+    wl = Syn.workload("1b_layer", Hq=14, Hkv=2, d=64, T=64, B=192)
+    _decode_case(wl, 6, 12, "bf16", n_streams=3)
+
+
+@cuda
+def test_decode_empty_detailed_state():
+    """No frame yet: the text attends to itself only (causal attention)."""
+    _decode_case(Syn.workload("8b_layer"), 0, 20, "bf16")
+
+
+@cuda
+def test_decode_8b_full_512_frames():
+    """The full 8B-class stream: decode 16 text tokens over all 131,072 video
+    tokens of D after 512 frames (the state the pages' generation reads)."""
+    _decode_case(Syn.workload("8b_layer"), 512, 16, "bf16", device_frames=True)
