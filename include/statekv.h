@@ -208,6 +208,14 @@ long long statekv_kernel_launches(statekv_t h);
  * that step are invalid).  Synchronises the device, then resets the word. */
 int statekv_device_status(statekv_t h, int* code);
 
+/* Time limit of the pipeline waits inside the handle's tensor-core kernels
+ * (ns <= 0 restores the default of 0.5 s).  A wait that runs past it makes
+ * the kernel record a code that statekv_device_status reports, drain its own
+ * copies and MMAs and exit; the results of that step are invalid, and later
+ * steps run normally.  Meant for testing that failure path: a limit of a few
+ * nanoseconds makes the waits give up on an otherwise healthy step. */
+int statekv_set_wait_limit(statekv_t h, long long ns);
+
 /* Frames processed so far on a layer (0 for a layer never called). */
 int statekv_frames(statekv_t h, int layer);
 

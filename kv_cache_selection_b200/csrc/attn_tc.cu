@@ -127,6 +127,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar_odone = [&](int x) { return sb + L::kBar + 8u * (5 + 2 * kSlots + x); };
   const uint32_t bar_done = sb + L::kBar + 8u * (7 + 2 * kSlots);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
+  const unsigned long long lim = a.wait_ns ? a.wait_ns : kWaitLimitNs;  // pipeline-wait limit
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
 
   if (threadIdx.x == 0) {
@@ -180,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int issued = 0;
       for (int idx = 0; idx < 2 * n_load; ++idx) {
         const int sl = idx % kSlots;
-        if (!mbar_wait(bar_kvempty(sl), ((idx / kSlots) & 1) ^ 1, a.err, kErrWaitEmpty, abort_flag)) break;
+        if (!mbar_wait(bar_kvempty(sl), ((idx / kSlots) & 1) ^ 1, a.err, kErrWaitEmpty, abort_flag, lim)) break;
         const int k = kb + (idx >> 1);
         const bool is_v = idx & 1;
         const bool is_c = k < a.nC;
@@ -212,7 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dv0 = sdesc_sw128(sb + L::kKV, L::kAtomBytes, 1024);
       auto slot16 = [&](int idx) { return (uint64_t)((idx % kSlots) * (L::kTileBytes >> 4)); };
       auto wait_slot = [&](int idx) {
-        return mbar_wait(bar_kvfull(idx % kSlots), (idx / kSlots) & 1, a.err, kErrWaitLoad, abort_flag);
+        return mbar_wait(bar_kvfull(idx % kSlots), (idx / kSlots) & 1, a.err, kErrWaitLoad, abort_flag, lim);
       };
       auto issue_s = [&](int x, int j) {  // S_x = Q_x K_j^T
         const uint64_t dq = dq0 + (uint64_t)((x * L::kTileBytes) >> 4), dk = dk0 + slot16(2 * j);
@@ -232,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ts(d_tmem, a_tmem + kk * 8, dv + (uint64_t)((kk * 2048) >> 4), id_o, (j > 0 || kk > 0) ? 1u : 0u);
         if (j == nX[x] - 1) mma_commit(bar_odone(x));
       };
-      bool ok = mbar_wait(bar_q, 0, a.err, kErrWaitLoad, abort_flag) && wait_slot(0);
+      bool ok = mbar_wait(bar_q, 0, a.err, kErrWaitLoad, abort_flag, lim) && wait_slot(0);
       if (ok) {
         fence_after_sync();
         if (nA > 0) issue_s(0, 0);
@@ -245,14 +246,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = wait_slot(2 * j + 1))) break;  // V_j
         const bool next_k = j + 1 < n_load;
         if (j < nA) {
-          if (!(ok = mbar_wait(bar_pfull(0), j & 1, a.err, kErrWaitP, abort_flag))) break;
+          if (!(ok = mbar_wait(bar_pfull(0), j & 1, a.err, kErrWaitP, abort_flag, lim))) break;
           fence_after_sync();
           issue_pv(0, j);
         }
         if (next_k && !(ok = wait_slot(2 * (j + 1)))) break;  // K_{j+1}
         if (j + 1 < nA) issue_s(0, j + 1);
         if (j < nB) {
-          if (!(ok = mbar_wait(bar_pfull(1), j & 1, a.err, kErrWaitP, abort_flag))) break;
+          if (!(ok = mbar_wait(bar_pfull(1), j & 1, a.err, kErrWaitP, abort_flag, lim))) break;
           fence_after_sync();
           issue_pv(1, j);
         }
@@ -283,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = ti.valid;
     for (int j = 0; ok && j < nX; ++j) {
       // S_j is on the critical chain: spin (a suspending wait wakes later)
-      if (!(ok = warp_spin_wait(bar_sfull(x), j & 1, a.err, kErrWaitAcc, abort_flag))) break;
+      if (!(ok = warp_spin_wait(bar_sfull(x), j & 1, a.err, kErrWaitAcc, abort_flag, lim))) break;
       fence_after_sync();
       const int k = kb + j;
       const bool is_c = k < a.nC;
@@ -361,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(bar_pfull(x));
     }
     // ---- epilogue: O / l and the row's log2-sum-exp
-    if (ok && nX > 0) ok = warp_wait(bar_odone(x), 0, a.err, kErrWaitAcc, abort_flag);
+    if (ok && nX > 0) ok = warp_wait(bar_odone(x), 0, a.err, kErrWaitAcc, abort_flag, lim);
     if (ok && ti.valid && !*abort_flag) {
       fence_after_sync();
       const bool row_ok = row_exists && i < a.T;

@@ -53,6 +53,7 @@ struct ScoreTcArgs {
   int m, T, Hq, Hkv, causal, n_c_tiles, n_f_tiles, S;
   float scale_log2;
   int* err;          // device error word (timeouts)
+  unsigned long long wait_ns;  // pipeline-wait limit; 0 = the default
 };
 cudaError_t launch_score_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kc, const CUtensorMap& tm_kf,
                             const ScoreTcArgs& a, int d, cudaStream_t st, bool pdl = false);
@@ -78,6 +79,7 @@ struct AttnTcArgs {
   int stack, q_rows;
   float scale_log2;
   int* err;
+  unsigned long long wait_ns;  // pipeline-wait limit; 0 = the default
 };
 int attn_tc_splits(int S, int Hq, int Hkv, int T, int m, int n_sm);
 cudaError_t launch_attn_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kc, const CUtensorMap& tm_vc,

@@ -55,6 +55,7 @@ struct statekv_handle {
   float* pool_score = nullptr;  // [S][Hkv][B+T]
   int32_t* idx = nullptr;       // [S][Hkv][max(B,1)]
   int* dev_err = nullptr;       // kernel error word (bounded-wait timeouts)
+  unsigned long long wait_ns = 0;  // pipeline-wait limit of the tensor-core kernels (0: default)
   __nv_bfloat16* o_part = nullptr;  // attention key-split partials (bf16 path)
   float* ml_part = nullptr;
   int max_split = 1;
@@ -478,6 +479,7 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
   ta.q_rows = 128;
     ta.scale_log2 = scale_log2;
     ta.err = h->dev_err;
+    ta.wait_ns = h->wait_ns;
     {
       StageScope sc(h, st, STATEKV_STAGE_ATTENTION);
       if ((e = skv::launch_attn_tc(tq, tkc, tvc, tkf, tvf, ta, d, st, true)) != cudaSuccess)
@@ -544,6 +546,7 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
     ta.S = S;
     ta.scale_log2 = scale_log2;
     ta.err = h->dev_err;
+    ta.wait_ns = h->wait_ns;
     StageScope sc(h, st, STATEKV_STAGE_SCORE);
     if ((e = skv::launch_score_tc(tq, tkc, tkf, ta, d, st, true)) != cudaSuccess) return launch_err(h, e, "score");
     sc.done();
@@ -735,6 +738,7 @@ int statekv_decode(statekv_t h, int layer, const void* q, const void* k, const v
   ta.nF = (n_text + 127) / 128;
   ta.scale_log2 = scale_log2;
   ta.err = h->dev_err;
+  ta.wait_ns = h->wait_ns;
   const int units = S * Hkv * ta.n_pairs;
   int split = std::max(1, h->n_sm / std::max(units, 1));
   split = std::min(split, std::min(ta.nC + ta.nF, 256));
@@ -875,6 +879,12 @@ int statekv_device_status(statekv_t h, int* code) {
   if (e == cudaSuccess) e = cudaMemset(h->dev_err, 0, sizeof(int));
   if (e != cudaSuccess) return set_err(h, STATEKV_ERR_CUDA, "status read failed: %s", cudaGetErrorString(e));
   *code = v;
+  return STATEKV_OK;
+}
+
+int statekv_set_wait_limit(statekv_t h, long long ns) {
+  if (!h) return set_err(nullptr, STATEKV_ERR_INVALID_ARG, "null handle");
+  h->wait_ns = ns > 0 ? (unsigned long long)ns : 0ull;
   return STATEKV_OK;
 }
 

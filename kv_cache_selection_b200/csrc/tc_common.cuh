@@ -2,10 +2,12 @@
 // tcgen05 tensor-memory allocation, MMA issue/commit, TMEM loads/stores and the
 // shared-memory / instruction descriptors of kind::f16 (bf16 in, f32 accumulate).
 //
-// Every wait is bounded in time: after kWaitLimitNs the waiting thread records
-// an error code in the kernel's error word, raises the CTA's abort flag and
-// returns false, so a kernel whose pipeline stalls exits (after draining its
-// own copies and MMAs and freeing its tensor memory) instead of hanging.
+// Every wait is bounded in time: after its limit (kWaitLimitNs unless the
+// caller passes another) the waiting thread records an error code in the
+// kernel's error word, raises the CTA's abort flag and returns false, so a
+// kernel whose pipeline stalls exits (after draining its own copies and MMAs,
+// waits bounded by kWaitLimitNs, and freeing its tensor memory) instead of
+// hanging.
 #pragma once
 
 #include <cuda.h>
@@ -67,14 +69,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // abort flag and the clock are checked every 64 polls only, so a waiting
 // thread takes few issue slots from the warps that share its scheduler.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err, int code,
-                                          volatile int* abort_flag) {
+                                          volatile int* abort_flag, unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         atomicCAS(err, 0, code);
         *abort_flag = 1;
         return false;
@@ -275,7 +277,7 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 // completed phase sooner than a suspending try_wait, at the cost of issue
 // slots, so it suits warps on the critical path.  The result is warp-uniform.
 __device__ __forceinline__ bool warp_spin_wait(uint32_t bar, uint32_t parity, int* err, int code,
-                                               volatile int* abort_flag) {
+                                               volatile int* abort_flag, unsigned long long limit_ns = kWaitLimitNs) {
   unsigned long long t0 = 0;
   for (uint32_t it = 0;; ++it) {
     if (__any_sync(0xffffffffu, mbar_test_wait(bar, parity))) return true;  // phases complete for good
@@ -286,7 +288,7 @@ __device__ __forceinline__ bool warp_spin_wait(uint32_t bar, uint32_t parity, in
           t0 = globaltimer_ns();
         } else if (*abort_flag) {
           stop = 1;
-        } else if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        } else if (globaltimer_ns() - t0 > limit_ns) {
           atomicCAS(err, 0, code);
           *abort_flag = 1;
           stop = 1;
@@ -299,9 +301,9 @@ __device__ __forceinline__ bool warp_spin_wait(uint32_t bar, uint32_t parity, in
 
 // Warp-uniform bounded wait: lane 0 polls, the result is broadcast.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int* err, int code,
-                                          volatile int* abort_flag) {
+                                          volatile int* abort_flag, unsigned long long limit_ns = kWaitLimitNs) {
   uint32_t ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, err, code, abort_flag) ? 1u : 0u;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, err, code, abort_flag, limit_ns) ? 1u : 0u;
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 

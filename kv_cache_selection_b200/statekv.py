@@ -50,6 +50,7 @@ _SIGS = {
     "statekv_profile_read": (_i, [_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)]),
     "statekv_kernel_launches": (ctypes.c_longlong, [_vp]),
     "statekv_device_status": (_i, [_vp, _ip]),
+    "statekv_set_wait_limit": (_i, [_vp, ctypes.c_longlong]),
     "statekv_destroy": (_i, [_vp]),
     "statekv_last_error": (ctypes.c_char_p, [_vp]),
     "statekv_step_noalloc": (_i, [_i] * 8 + [_vp] * 7 + [_i] + [_vp] * 8 + [_i, _i, _vp]),
@@ -181,6 +182,10 @@ class StateKV:
         code = ctypes.c_int()
         _check(lib.statekv_device_status(self._h, ctypes.byref(code)), self._h)
         return code.value
+
+    def set_wait_limit(self, ns: int):
+        """Pipeline-wait limit of the tensor-core kernels (<= 0: the default)."""
+        _check(lib.statekv_set_wait_limit(self._h, int(ns)), self._h)
 
     def kernel_launches(self) -> int:
         return lib.statekv_kernel_launches(self._h)

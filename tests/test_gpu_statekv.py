@@ -526,3 +526,44 @@ def test_decode_8b_full_512_frames():
     """The full 8B-class stream: decode 16 text tokens over all 131,072 video
     tokens of D after 512 frames (the state the pages' generation reads)."""
     _decode_case(Syn.workload("8b_layer"), 512, 16, "bf16", device_frames=True)
+
+
+@cuda
+def test_pipeline_wait_timeout_is_reported_and_recovers():
+    """Failure path of the tensor-core kernels, made to happen without a GPU
+    fault: with a pipeline-wait limit of 1 ns the waits give up, record their
+    code in the handle's device status word, drain their own copies and MMAs
+    and exit.  The status reports it; with the default limit restored the next
+    steps are correct again (checked against the oracle from the GPU's own
+    compressed state) and report no error."""
+    S = _skv()
+    wl = Syn.workload("1b_layer", Hq=14, Hkv=2, d=64, T=128, B=256, frames=6)
+    dev = torch.device("cuda")
+    h = S.StateKV(wl.Hq, wl.Hkv, wl.d, wl.T, wl.B, max_frames=wl.frames, dtype="bf16")
+    frames = [tuple(t.to(dev) for t in Syn.gen_frame(wl, n)) for n in range(wl.frames)]
+    for n in range(2):
+        h.prefill_frame(0, *frames[n])
+    assert h.device_status() == 0
+    h.set_wait_limit(1)
+    codes = []
+    for n in range(2, 4):
+        h.prefill_frame(0, *frames[n])
+        codes.append(h.device_status())
+    assert any(c in (1, 2, 3, 4, 5) for c in codes), codes   # a pipeline wait gave up
+    assert all(c in (0, 1, 2, 3, 4, 5) for c in codes), codes
+    h.set_wait_limit(0)
+    for n in range(4, 6):
+        C_before = _clone_C(h.get_compressed(0))
+        out = h.prefill_frame(0, *frames[n])
+        torch.cuda.synchronize()
+        st = P.oracle_state_from_gpu(C_before)
+        q, k, v, pos = (t.cpu() for t in frames[n])
+        _, res = O.statekv_step(st, q, k, v, pos.numpy(), wl.B)
+        P.check_out(out, res["out"], "bf16", what=f"frame {n} after the timeout")
+        stats = h.step_stats()
+        P.check_lse(stats["lse"][0], res["lse"], "bf16")
+        C = h.get_compressed(0)
+        P.check_selection(C["pos"][0, 0, :C["len"]].cpu().numpy(), res["kept"][0], res["score"][0],
+                          res["pool_pos"][0], wl.B)
+    assert h.device_status() == 0
+    h.close()
