@@ -544,31 +544,81 @@ def run_diagnostics(args):
 
 
 def run_stack(args):
-    """28 independent 8B-class layers, layers in order per frame, 128 frames."""
+    """28 independent 8B-class layers over 128 frames.  In-order schedule:
+    every frame runs its layers in order on one stream (per-frame latency vs
+    frame index).  Pipelined schedule: frames alternate over `--stack-pipeline`
+    streams and layer l of frame n+1 waits only for layer l of frame n (an
+    event per layer), so frame n+1's early layers overlap frame n's later
+    ones; reported as frames/s per layer over the same frames."""
     from kv_cache_selection_b200 import statekv as SKV
     wl = Syn.workload("8b_stack")
     dev = torch.device("cuda")
     n_frames = args.stack_frames or wl.frames
     layers = [Syn.gen_frames_device(wl, n_frames, layer=l, device=dev) for l in range(wl.layers)]
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.int32, device=dev)
+    fill = math.ceil(wl.B / wl.T)
+    d_bytes = wl.layers * n_frames * wl.T * wl.Hkv * wl.d * 2 * 2
+
+    # in order, one stream, per-frame events
     h = SKV.StateKV(wl.Hq, wl.Hkv, wl.d, wl.T, wl.B, max_frames=n_frames, dtype=wl.dtype)
     h.reserve_layers(wl.layers)
     out = torch.empty_like(layers[0][0][0])
-    flush = torch.empty(64 * 1024 * 1024, dtype=torch.int32, device=dev)
 
     def frame(n):
         for l, (q, k, v, pos) in enumerate(layers):
             h.prefill_frame(l, q[n], k[n], v[n], pos[n], out)
 
     us = _per_frame_times(frame, n_frames, flush, dev)
-    fill = math.ceil(wl.B / wl.T)
-    d_bytes = wl.layers * n_frames * wl.T * wl.Hkv * wl.d * 2 * 2
-    rep = {"report": "stack", "workload": f"8b_stack: {wl.layers} layers x {n_frames} frames, B={wl.B}",
-           "per_frame_us_all_layers": _flatness(us, fill),
-           "per_frame_layer_us": round(_flatness(us, fill)["p50_us"] / wl.layers, 2),
-           "frames_per_s_per_layer": round(1e6 / (_flatness(us, fill)["p50_us"] / wl.layers), 1),
-           "detailed_state_bytes_K_plus_V": d_bytes,
-           "per_frame_us_every_8": [round(x, 1) for x in us[::8]]}
     h.close()
+    flat = _flatness(us, fill)
+    rep = {"report": "stack", "workload": f"8b_stack: {wl.layers} layers x {n_frames} frames, B={wl.B}",
+           "in_order": {"per_frame_us_all_layers": flat,
+                        "per_frame_layer_us": round(flat["p50_us"] / wl.layers, 2),
+                        "frames_per_s_per_layer": round(1e6 / (flat["p50_us"] / wl.layers), 1),
+                        "per_frame_us_every_8": [round(x, 1) for x in us[::8]]},
+           "detailed_state_bytes_K_plus_V": d_bytes}
+
+    # whole-run throughput of the steady-state frames, L2 not flushed (frames
+    # overlap in the pipelined schedule): one stream (in order) against P
+    # streams (pipelined)
+    main = torch.cuda.current_stream()
+
+    def whole_run(P):
+        h = SKV.StateKV(wl.Hq, wl.Hkv, wl.d, wl.T, wl.B, max_frames=n_frames, dtype=wl.dtype)
+        h.reserve_layers(wl.layers)
+        streams = [torch.cuda.Stream(device=dev) for _ in range(P)]
+        outs = [torch.empty_like(out) for _ in range(P)]
+        layer_done = [torch.cuda.Event() for _ in range(wl.layers)]
+
+        def run_frames(n0, n1):
+            for n in range(n0, n1):
+                st = streams[n % P]
+                for l, (q, k, v, pos) in enumerate(layers):
+                    st.wait_event(layer_done[l])          # frame n-1 of layer l is done
+                    h.prefill_frame(l, q[n], k[n], v[n], pos[n], outs[n % P], stream=st)
+                    layer_done[l].record(st)
+
+        for st in streams:
+            st.wait_stream(main)
+        run_frames(0, fill)                               # fill C (not timed)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(main)
+        for st in streams:
+            st.wait_stream(main)
+        run_frames(fill, n_frames)
+        for st in streams:
+            main.wait_stream(st)
+        e1.record(main)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+        h.close()
+        steady = n_frames - fill
+        return {"streams": P, "frames_timed": steady, "per_frame_us_all_layers": round(ms * 1e3 / steady, 1),
+                "per_frame_layer_us": round(ms * 1e3 / steady / wl.layers, 2),
+                "frames_per_s_per_layer": round(steady * wl.layers / (ms / 1e3), 1)}
+
+    rep["whole_run_unflushed"] = {"in_order": whole_run(1), "pipelined": whole_run(max(2, args.stack_pipeline))}
     return rep
 
 
@@ -715,6 +765,7 @@ def main(argv=None):
     ap.add_argument("--mode", choices=["headline", "flatness", "stack", "sweep", "diagnostics"], default="headline",
                     help="headline: the contract's JSON line; others: report lines")
     ap.add_argument("--stack-frames", type=int, default=0)
+    ap.add_argument("--stack-pipeline", type=int, default=2, help="streams of the pipelined stack schedule")
     ap.add_argument("--diag-frames", type=int, default=64)
     ap.add_argument("--diag-b", type=int, default=1024, help="budget of the retained sets compared")
     ap.add_argument("--diag-budgets", type=int, nargs="+", default=[1, 16, 256, 1024, 4096])

@@ -73,7 +73,7 @@ typedef enum {
 } statekv_status;
 
 /* Create a handle for one video stream (S = 1).
- * Allocates per-step scratch now; per-layer state (C and D) is allocated on a
+ * Per-layer state (C, D and the layer's own step scratch) is allocated on a
  * layer's first prefill_frame call (or by statekv_reserve_layers).
  * max_frames bounds the frames per layer (D holds max_frames*T tokens).
  * B >= 0 (B = 0: no cross-frame context).  Errors: INVALID_ARG, UNSUPPORTED,
@@ -108,9 +108,13 @@ int statekv_reserve_layers(statekv_t h, int n_layers);
  *                       ascending and above all earlier frames' positions.
  *                       The library stores them and never re-rotates.
  * Output (device pointer): out [S][T][Hq][d] (dtype).
- * Frame n of a layer must follow frame n-1 of that layer on the same stream
- * order; layers may interleave.  Errors: INVALID_ARG, CAPACITY, OOM (first use
- * of a layer), CUDA. */
+ * Frame n of a layer must follow frame n-1 of that layer in stream order;
+ * layers may interleave.  Steps of different layers share no device memory
+ * (each layer has its own C, D and step scratch), so they may also run
+ * concurrently on different streams, e.g. frame n+1 of layer l beside frame n
+ * of layer l+1 (order each layer's frames with events).  Calls on one handle
+ * must come from one host thread at a time.  Errors: INVALID_ARG, CAPACITY,
+ * OOM (first use of a layer), CUDA. */
 int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k,
                           const void* v, const int32_t* pos, void* out, void* stream);
 
@@ -164,13 +168,15 @@ int statekv_get_compressed(statekv_t h, int layer, const void** k, const void** 
 int statekv_get_detailed(statekv_t h, int layer, const void** k, const void** v,
                          const int32_t** pos, int* len);
 
-/* Borrow the per-row statistics of the most recent prefill_frame (any layer):
+/* Borrow the per-row statistics of the most recent prefill_frame call (of
+ * whichever layer it was):
  *   lse        [S][Hq][T] float32, natural-log log-sum-exp of each query row;
  *   pool_score [S][Hkv][B+T] float32, the score of every pool candidate
  *              (C entries first, then frame tokens); entries [0, pool_len)
  *              valid.  In GLOBAL and RECENCY modes only row 0 of each stream
  *              is written.
- * Valid until the next prefill_frame.  Any output pointer may be NULL. */
+ * Valid until the next prefill_frame on that layer.  Any output pointer may be
+ * NULL.  Errors: INVALID_ARG (no step has run yet). */
 int statekv_get_step_stats(statekv_t h, const float** lse, const float** pool_score,
                            int* pool_len);
 
@@ -288,6 +294,14 @@ int statekv_step_noalloc(int Hq, int Hkv, int d, int T, int B, int dtype, int ma
                          const int32_t* posc, int m, void* out, void* kc_new, void* vc_new,
                          int32_t* posc_new, float* scorec_new, void* kd, void* vd,
                          int32_t* posd, int d_len, int max_tok, void* stream);
+
+/* Self-test of the FMA-pipe exponential the kernels may use in place of the
+ * MUFU unit for part of their exponentials: y[i] = 2^x[i] for n float32
+ * values (device pointers) on `stream`.  The paper has no counterpart; tests
+ * compare it with CUDA's exp2f (maximum relative error 7.5e-5 for
+ * -125 <= x <= 127; below -125 a non-negative value under 2^-124).  Errors (message in statekv_last_error(NULL)):
+ * INVALID_ARG, CUDA. */
+int statekv_selftest_exp2(const float* x, float* y, int n, void* stream);
 
 #ifdef __cplusplus
 }

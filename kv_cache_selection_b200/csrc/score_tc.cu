@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar_accempty = [&](int b) { return sb + L::kBar + 8u * (5 + 2 * kStages + b); };
   const uint32_t bar_done = sb + L::kBar + 8u * (9 + 2 * kStages);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
-  const unsigned long long lim = a.wait_ns ? a.wait_ns : kWaitLimitNs;  // pipeline-wait limit
+  const unsigned long long wait_lim = a.wait_ns ? a.wait_ns : kWaitLimitNs;  // pipeline-wait limit
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
 
   if (threadIdx.x == 0) {
@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int issued = 0;
       for (int c = 0; c < n_chunks; ++c) {
         const int st = c % kStages;
-        if (!mbar_wait(bar_qempty(st), ((c / kStages) & 1) ^ 1, a.err, kErrWaitEmpty, abort_flag, lim)) break;
+        if (!mbar_wait(bar_qempty(st), ((c / kStages) & 1) ^ 1, a.err, kErrWaitEmpty, abort_flag, wait_lim)) break;
         const int h = g * G + c / per_head;
         const int i0 = (ic_min + c % per_head) * 128;
         mbar_arrive_expect_tx(bar_qfull(st), L::kTileBytes);
@@ -170,11 +170,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(128, 128, false, false);
-      bool ok = mbar_wait(bar_k, 0, a.err, kErrWaitLoad, abort_flag, lim);
+      bool ok = mbar_wait(bar_k, 0, a.err, kErrWaitLoad, abort_flag, wait_lim);
       for (int c = 0; ok && c < n_chunks; ++c) {
         const int st = c % kStages, buf = c & 3;
-        if (!mbar_wait(bar_qfull(st), (c / kStages) & 1, a.err, kErrWaitLoad, abort_flag, lim)) break;
-        if (!mbar_wait(bar_accempty(buf), ((c >> 2) & 1) ^ 1, a.err, kErrWaitAccFree, abort_flag, lim)) break;
+        if (!mbar_wait(bar_qfull(st), (c / kStages) & 1, a.err, kErrWaitLoad, abort_flag, wait_lim)) break;
+        if (!mbar_wait(bar_accempty(buf), ((c >> 2) & 1) ^ 1, a.err, kErrWaitAccFree, abort_flag, wait_lim)) break;
         fence_after_sync();
         const uint32_t qbase = sb + L::kQ + st * L::kTileBytes;
 #pragma unroll
@@ -246,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int i0 = (ic_min + c % per_head) * 128;
       const float* lse2 = lse_all + hh * tpad + i0;
       uint32_t got = 1;
-      if (lane == 0) got = mbar_wait(bar_accfull(buf), (c >> 2) & 1, a.err, kErrWaitAcc, abort_flag, lim) ? 1u : 0u;
+      if (lane == 0) got = mbar_wait(bar_accfull(buf), (c >> 2) & 1, a.err, kErrWaitAcc, abort_flag, wait_lim) ? 1u : 0u;
       got = __shfl_sync(0xffffffffu, got, 0);
       if (!got) {
         ok = false;

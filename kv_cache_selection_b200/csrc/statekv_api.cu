@@ -38,6 +38,15 @@ struct LayerState {
   void* kd = nullptr;
   void* vd = nullptr;
   int32_t* posd = nullptr;
+  // per-step scratch of this layer (each layer has its own, so that steps of
+  // different layers may run concurrently on different streams)
+  float* lse = nullptr;         // [S][Hq][T]
+  float* part = nullptr;        // [S][Hkv][B+T]
+  float* pool_score = nullptr;  // [S][Hkv][B+T]
+  int32_t* idx = nullptr;       // [S][Hkv][max(B,1)]
+  __nv_bfloat16* o_part = nullptr;  // attention key-split partials (bf16 path)
+  float* ml_part = nullptr;
+  int pool_len = 0;             // pool size of the layer's last step
 };
 
 }  // namespace
@@ -49,16 +58,10 @@ struct statekv_handle {
   int device = 0;
   size_t esize = 2;
   std::vector<LayerState> layers;
-  // per-step scratch
-  float* lse = nullptr;         // [S][Hq][T]
-  float* part = nullptr;        // [S][Hkv][B+T]
-  float* pool_score = nullptr;  // [S][Hkv][B+T]
-  int32_t* idx = nullptr;       // [S][Hkv][max(B,1)]
   int* dev_err = nullptr;       // kernel error word (bounded-wait timeouts)
   unsigned long long wait_ns = 0;  // pipeline-wait limit of the tensor-core kernels (0: default)
-  __nv_bfloat16* o_part = nullptr;  // attention key-split partials (bf16 path)
-  float* ml_part = nullptr;
-  int max_split = 1;
+  int max_split = 1;            // key splits the attention scratch is sized for
+  int last_layer = -1;          // layer of the most recent prefill_frame
   // statekv_prefill_frame_host: two staging sets used in turn, a copy stream
   // for the host-to-device copies, and the events that order them (created on
   // first use)
@@ -71,7 +74,6 @@ struct statekv_handle {
   cudaStream_t copy_stream = nullptr;
   cudaEvent_t ev_h2d[2] = {nullptr, nullptr};   // inputs of set b are on the device
   cudaEvent_t ev_stage_free[2] = {nullptr, nullptr};  // the step and copy-out of set b are done
-  int last_pool_len = 0;
   // key-split partials of statekv_decode (float32), grown on demand
   float* dec_o = nullptr;
   float* dec_ml = nullptr;
@@ -159,6 +161,16 @@ int alloc_layer(statekv_t h, LayerState& L) {
   if ((rc = dev_alloc(h, &L.kd, dbytes))) return rc;
   if ((rc = dev_alloc(h, &L.vd, dbytes))) return rc;
   if ((rc = dev_alloc(h, (void**)&L.posd, (size_t)h->S * max_tok * 4))) return rc;
+  const size_t S = h->S, pool = (size_t)h->B + h->T;
+  if ((rc = dev_alloc(h, (void**)&L.lse, S * h->Hq * h->T * 4)) ||
+      (rc = dev_alloc(h, (void**)&L.part, S * h->Hkv * pool * 4)) ||
+      (rc = dev_alloc(h, (void**)&L.pool_score, S * h->Hkv * pool * 4)) ||
+      (rc = dev_alloc(h, (void**)&L.idx, S * h->Hkv * std::max(h->B, 1) * 4)))
+    return rc;
+  if (h->max_split > 1 &&
+      ((rc = dev_alloc(h, (void**)&L.o_part, S * h->Hq * h->max_split * h->T * h->d * 2)) ||
+       (rc = dev_alloc(h, (void**)&L.ml_part, S * h->Hq * h->max_split * h->T * 4))))
+    return rc;
   L.ready = true;
   return STATEKV_OK;
 }
@@ -366,26 +378,12 @@ int statekv_create_batched(statekv_t* out, int n_streams, int Hq, int Hkv, int d
     delete h;
     return STATEKV_ERR_CUDA;
   }
-  const size_t pool = (size_t)B + T;
-  if ((rc = dev_alloc(h, (void**)&h->lse, (size_t)n_streams * Hq * T * 4)) ||
-      (rc = dev_alloc(h, (void**)&h->part, (size_t)n_streams * Hkv * pool * 4)) ||
-      (rc = dev_alloc(h, (void**)&h->pool_score, (size_t)n_streams * Hkv * pool * 4)) ||
-      (rc = dev_alloc(h, (void**)&h->idx, (size_t)n_streams * Hkv * std::max(B, 1) * 4)) ||
-      (rc = dev_alloc(h, (void**)&h->dev_err, 16))) {
+  if ((rc = dev_alloc(h, (void**)&h->dev_err, 16))) {
     g_free_error = h->err;
     statekv_destroy(h);
     return rc;
   }
-  if (dtype == STATEKV_BF16) {
-    h->max_split = skv::attn_tc_splits(n_streams, Hq, Hkv, T, B, h->n_sm);
-    if (h->max_split > 1 &&
-        ((rc = dev_alloc(h, (void**)&h->o_part, (size_t)n_streams * Hq * h->max_split * T * d * 2)) ||
-         (rc = dev_alloc(h, (void**)&h->ml_part, (size_t)n_streams * Hq * h->max_split * T * 4)))) {
-      g_free_error = h->err;
-      statekv_destroy(h);
-      return rc;
-    }
-  }
+  if (dtype == STATEKV_BF16) h->max_split = skv::attn_tc_splits(n_streams, Hq, Hkv, T, B, h->n_sm);
   *out = h;
   return STATEKV_OK;
 }
@@ -444,7 +442,7 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
   aa.b_row = Hkv * d;
   aa.nb = T;
   aa.out = out;
-  aa.lse = h->lse;
+  aa.lse = L->lse;
   aa.lse_s = (long long)Hq * T;
   aa.n_rows = T;
   aa.Hq = Hq;
@@ -460,10 +458,10 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
     ta.out = out;
     ta.out_s = (long long)T * Hq * d;
     ta.out_row = Hq * d;
-    ta.lse = h->lse;
+    ta.lse = L->lse;
     ta.lse_s = (long long)Hq * T;
-    ta.o_part = h->o_part;
-    ta.ml_part = h->ml_part;
+    ta.o_part = L->o_part;
+    ta.ml_part = L->ml_part;
     ta.m = m;
     ta.T = T;
     ta.Hq = Hq;
@@ -517,9 +515,9 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
   sa.b_s = aa.b_s;
   sa.b_row = aa.b_row;
   sa.nb = T;
-  sa.lse = h->lse;
+  sa.lse = L->lse;
   sa.lse_s = aa.lse_s;
-  sa.part = h->part;
+  sa.part = L->part;
   sa.part_s = (long long)Hkv * pool;
   sa.part_g = pool;
   sa.n_rows = T;
@@ -529,11 +527,11 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
   sa.scale_log2 = scale_log2;
   if (h->dtype == STATEKV_BF16) {
     skv::ScoreTcArgs ta{};
-    ta.lse = h->lse;
+    ta.lse = L->lse;
     ta.lse_s = aa.lse_s;
-    ta.ml_part = h->ml_part;
+    ta.ml_part = L->ml_part;
     ta.n_split = n_split;
-    ta.part = h->part;
+    ta.part = L->part;
     ta.part_s = sa.part_s;
     ta.part_g = pool;
     ta.m = m;
@@ -558,13 +556,13 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
 
   // (c) top-B select
   skv::SelectArgs se{};
-  se.part = h->part;
+  se.part = L->part;
   se.part_s = sa.part_s;
   se.part_g = pool;
-  se.pool_score = h->pool_score;
+  se.pool_score = L->pool_score;
   se.pos_c = L->posc[cur];
   se.pos_f = pos;
-  se.idx = h->idx;
+  se.idx = L->idx;
   se.Hkv = Hkv;
   se.m = m;
   se.T = T;
@@ -586,7 +584,7 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
   ga.vf = v;
   ga.kc_new = L->kc[nxt];
   ga.vc_new = L->vc[nxt];
-  ga.idx = h->idx;
+  ga.idx = L->idx;
   ga.kd = L->kd;
   ga.vd = L->vd;
   ga.pos_d = L->posd;
@@ -615,7 +613,8 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
   L->m = m_new;
   L->cur = nxt;
   L->frames += 1;
-  h->last_pool_len = m + T;
+  L->pool_len = m + T;
+  h->last_layer = layer;
   return STATEKV_OK;
 }
 
@@ -826,9 +825,11 @@ int statekv_get_detailed(statekv_t h, int layer, const void** k, const void** v,
 
 int statekv_get_step_stats(statekv_t h, const float** lse, const float** pool_score, int* pool_len) {
   if (!h) return set_err(nullptr, STATEKV_ERR_INVALID_ARG, "null handle");
-  if (lse) *lse = h->lse;
-  if (pool_score) *pool_score = h->pool_score;
-  if (pool_len) *pool_len = h->last_pool_len;
+  if (h->last_layer < 0) return set_err(h, STATEKV_ERR_INVALID_ARG, "no step has run yet");
+  const LayerState& L = h->layers[h->last_layer];
+  if (lse) *lse = L.lse;
+  if (pool_score) *pool_score = L.pool_score;
+  if (pool_len) *pool_len = L.pool_len;
   return STATEKV_OK;
 }
 
