@@ -292,9 +292,13 @@ def run_ours(args, wl):
     torch.cuda.synchronize()
 
     # ---- flatness: the full 512-frame stream of the 8B layer, per-frame time
-    flat = dec = None
+    flat = dec = cross = None
     if not args.no_flatness and wl.name == "8b_layer":
         flat, dec = flatness_report(SKV, wl, dev)
+        cs = ClockSampler(local_rank)
+        cs.start()
+        cross = sweep_report([32, 64, 128, 256], [4096], dev)
+        cross["clocks"] = cs.stop()
 
     if rank != 0:
         h.close()
@@ -363,7 +367,7 @@ def run_ours(args, wl):
         "step_us_p99": round(sorted(ms_steps)[int(0.99 * (len(ms_steps) - 1))] * 1e3, 2),
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
         "gpu_launches_per_step": launches / K, "host_enqueue_us_per_step": round(host_enqueue_us, 2),
-        "clocks": clk, "flatness": flat, "decode": dec,
+        "clocks": clk, "flatness": flat, "decode": dec, "crossover": cross,
     }
     print(json.dumps(line), flush=True)
 
@@ -396,11 +400,26 @@ def cpu_baseline(wl, h, fr_cpu, n_next, n_distinct, budget_s=20.0, kv_heads=None
     threads = [p.get("num_threads", 1) for p in threadpool_info() if p.get("user_api") == "blas"]
     frac = kvh / wl.Hkv
     value = frames_done * frac / el
+    # the same oracle restricted to one BLAS thread, on a few more frames
+    from threadpoolctl import threadpool_limits
+    one_frames, t1 = 0, time.perf_counter()
+    with threadpool_limits(limits=1):
+        while True:
+            q, k, v, _ = fr_cpu[n % n_distinct]
+            pos = torch.arange(n * wl.T, (n + 1) * wl.T).numpy()
+            st, _ = O.statekv_step(st, q[:, :kvh * G], k[:, :kvh], v[:, :kvh], pos, wl.B)
+            one_frames += 1
+            n += 1
+            el1 = time.perf_counter() - t1
+            if el1 > budget_s / 4 or one_frames >= 8:
+                break
     return {"value": round(value, 5), "unit": UNIT, "cores": int(max(threads) if threads else 1),
             "host_cpus": os.cpu_count(), "kind": "oracle",
+            "value_1_core": round(one_frames * frac / el1, 5),
             "sample": f"{frames_done} steady-state frames of {wl.name} on {kvh} of {wl.Hkv} KV heads "
                       f"({kvh * G} query heads), float64 numpy oracle, {el:.1f} s; value scaled by "
-                      f"{wl.Hkv}/{kvh}"}
+                      f"{wl.Hkv}/{kvh}; value_1_core: {one_frames} further frames with one BLAS thread, "
+                      f"{el1:.1f} s"}
 
 
 # ------------------------------------------------------------ report modes --
@@ -622,14 +641,15 @@ def run_stack(args):
     return rep
 
 
-def run_sweep(args):
-    """8B layer shape, 4 streams per launch: cumulative StateKV prefill cost
-    against full_causal_prefill over the same N*256 tokens."""
+def sweep_report(frames_list, b_list, dev):
+    """8B layer shape, 4 streams per launch: cumulative StateKV prefill device
+    time over the first N frames against full_causal_prefill over the same
+    N*256 tokens (one batched call, 4 sequences), and the first N on the grid
+    where StateKV is cheaper (the compute crossover)."""
     from kv_cache_selection_b200 import statekv as SKV
     wl = Syn.workload("8b_sweep")
-    dev = torch.device("cuda")
     S = wl.streams
-    n_max = max(args.sweep_frames)
+    n_max = max(frames_list)
     per = [Syn.gen_frames_device(wl, n_max, stream=s, device=dev) for s in range(S)]
     # [S][n][T][H][d] so that the first N frames of a stream are one sequence
     Q = torch.stack([p[0] for p in per])
@@ -638,10 +658,10 @@ def run_sweep(args):
     P = torch.stack([p[3] for p in per])
     del per
     flush = torch.empty(64 * 1024 * 1024, dtype=torch.int32, device=dev)
-    res = {"report": "sweep", "workload": f"8b layer shape, {S} streams per launch, frames {args.sweep_frames}",
+    res = {"workload": f"8b layer shape, {S} streams per launch, frames {list(frames_list)}",
            "statekv": {}, "full_causal_us": {}, "crossover_frames": {}, "analytic_crossover_frames_3_passes": {}}
     fc = {}
-    for N in args.sweep_frames:
+    for N in frames_list:
         ntok = N * wl.T
         q = Q[:, :N].reshape(S, ntok, wl.Hq, wl.d).contiguous()
         kk = Kt[:, :N].reshape(S, ntok, wl.Hkv, wl.d).contiguous()
@@ -658,7 +678,7 @@ def run_sweep(args):
         fc[N] = e0.elapsed_time(e1) * 1e3
         res["full_causal_us"][N] = round(fc[N], 1)
         del out, q, kk, vv
-    for B in args.sweep_b:
+    for B in b_list:
         h = SKV.StateKV(wl.Hq, wl.Hkv, wl.d, wl.T, B, max_frames=n_max, dtype=wl.dtype, n_streams=S)
         h.reserve_layers(1)
         qs = torch.empty((S, wl.T, wl.Hq, wl.d), dtype=wl.torch_dtype, device=dev)
@@ -680,19 +700,24 @@ def run_sweep(args):
         cum, acc = {}, 0.0
         for n, t in enumerate(us):
             acc += t
-            if n + 1 in args.sweep_frames:
+            if n + 1 in frames_list:
                 cum[n + 1] = round(acc, 1)
         fill = math.ceil(B / wl.T)
         res["statekv"][B] = {"cumulative_us": cum, "steady_step_us_4_streams": _flatness(us, fill)["p50_us"]}
         cross = None
-        for N in sorted(args.sweep_frames):
+        for N in sorted(frames_list):
             if cum[N] <= fc[N]:
                 cross = N
                 break
         res["crossover_frames"][B] = cross
         res["analytic_crossover_frames_3_passes"][B] = round(3 * (B + wl.T / 2) / wl.T, 1)
         h.close()
+    del Q, Kt, V, P
     return res
+
+
+def run_sweep(args):
+    return dict(report="sweep", **sweep_report(args.sweep_frames, args.sweep_b, torch.device("cuda")))
 
 
 # ------------------------------------------------------------ reference arm --

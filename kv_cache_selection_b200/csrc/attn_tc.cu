@@ -551,13 +551,13 @@ cudaError_t launch_attn_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kc, co
   cudaError_t e;
   if (d == 128) {
     const int smem = AttnSmem<128>::kAlloc;
-    if ((e = cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)))
+    if ((e = ensure_dynamic_smem(attn_tc_kernel<128>, smem)))
       return e;
     return launch_kernel(attn_tc_kernel<128>, dim3(units), dim3(kThreads), smem, st, pdl, tm_q, tm_kc, tm_vc,
                          tm_kf, tm_vf, a);
   } else {
     const int smem = AttnSmem<64>::kAlloc;
-    if ((e = cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)))
+    if ((e = ensure_dynamic_smem(attn_tc_kernel<64>, smem)))
       return e;
     return launch_kernel(attn_tc_kernel<64>, dim3(units), dim3(kThreads), smem, st, pdl, tm_q, tm_kc, tm_vc,
                          tm_kf, tm_vf, a);

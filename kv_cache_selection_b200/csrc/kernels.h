@@ -26,6 +26,15 @@ cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
+// Raise a kernel's dynamic shared-memory limit on the current device to at
+// least `bytes`, calling the driver only when the recorded limit is lower
+// (the attribute persists for the process).
+cudaError_t ensure_dynamic_smem(const void* kernel, int bytes);
+template <typename... KArgs>
+cudaError_t ensure_dynamic_smem(void (*kernel)(KArgs...), int bytes) {
+  return ensure_dynamic_smem(reinterpret_cast<const void*>(kernel), bytes);
+}
+
 constexpr int kDtypeBF16 = 0;
 constexpr int kDtypeF32 = 1;
 

@@ -29,6 +29,9 @@ namespace {
 using namespace tc;
 
 constexpr int kStages = 4;
+// Every kFmaExpEvery-th exponential runs on the FMA pipe (exp2_fma) instead of
+// MUFU, which otherwise issues all of them (0: none).
+constexpr int kFmaExpEvery = 0;
 constexpr int kGroups = 3;                      // epilogue warpgroups (take chunks round robin)
 constexpr int kEpiWarps = 4 * kGroups;
 constexpr int kThreads = 128 + 32 * kEpiWarps;  // warpgroup 0: producer, MMA, two idle warps
@@ -65,10 +68,14 @@ __device__ __forceinline__ void score_cols16(const uint32_t (&rr)[16], const flo
 #pragma unroll
   for (int j4 = 0; j4 < 4; ++j4) {
     const float4 lv = l4[j4];  // -lse2 of 4 columns
-    float p0 = ex2_approx(fmaf(__uint_as_float(rr[4 * j4 + 0]), scale_log2, lv.x));
-    float p1 = ex2_approx(fmaf(__uint_as_float(rr[4 * j4 + 1]), scale_log2, lv.y));
-    float p2 = ex2_approx(fmaf(__uint_as_float(rr[4 * j4 + 2]), scale_log2, lv.z));
-    float p3 = ex2_approx(fmaf(__uint_as_float(rr[4 * j4 + 3]), scale_log2, lv.w));
+    auto ex = [](int e, float x) {
+      return (kFmaExpEvery > 0 && e % (kFmaExpEvery > 0 ? kFmaExpEvery : 1) == kFmaExpEvery - 1) ? exp2_fma(x)
+                                                                                              : ex2_approx(x);
+    };
+    float p0 = ex(4 * j4 + 0, fmaf(__uint_as_float(rr[4 * j4 + 0]), scale_log2, lv.x));
+    float p1 = ex(4 * j4 + 1, fmaf(__uint_as_float(rr[4 * j4 + 1]), scale_log2, lv.y));
+    float p2 = ex(4 * j4 + 2, fmaf(__uint_as_float(rr[4 * j4 + 2]), scale_log2, lv.z));
+    float p3 = ex(4 * j4 + 3, fmaf(__uint_as_float(rr[4 * j4 + 3]), scale_log2, lv.w));
     if (need_mask) {
       // frame token `key` is seen by rows i >= key (frame-causal); rows past T do not exist
       const int i = i0 + 4 * j4;
@@ -315,12 +322,12 @@ cudaError_t launch_score_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kc, c
   const int lse_bytes = (a.Hq / a.Hkv) * n_ic * 128 * 4;
   if (d == 128) {
     const int smem = Smem<128>::kAlloc + lse_bytes;
-    if ((e = cudaFuncSetAttribute(score_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)))
+    if ((e = ensure_dynamic_smem(score_tc_kernel<128>, smem)))
       return e;
     return launch_kernel(score_tc_kernel<128>, grid, dim3(kThreads), smem, st, pdl, tm_q, tm_kc, tm_kf, a);
   } else {
     const int smem = Smem<64>::kAlloc + lse_bytes;
-    if ((e = cudaFuncSetAttribute(score_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)))
+    if ((e = ensure_dynamic_smem(score_tc_kernel<64>, smem)))
       return e;
     return launch_kernel(score_tc_kernel<64>, grid, dim3(kThreads), smem, st, pdl, tm_q, tm_kc, tm_kf, a);
   }

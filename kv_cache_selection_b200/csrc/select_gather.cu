@@ -459,8 +459,7 @@ cudaError_t launch_select(const SelectArgs& a_in, int S, cudaStream_t st, bool p
   // the default 48 KB per block covers static and dynamic shared memory
   // together; the kernel's static arrays take ~19 KB, so opt in above 24 KB
   if (smem > 24 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(select_topb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    cudaError_t e = ensure_dynamic_smem(select_topb_kernel, (int)smem);
     if (e != cudaSuccess) return e;
   }
   return launch_kernel(select_topb_kernel, dim3(a.n_sel_blocks + a.n_mrg_blocks), dim3(kSelThreads), smem, st,

@@ -1,10 +1,12 @@
-// Host-side encoding of TMA tensor maps (cuTensorMapEncodeTiled through the
-// runtime's driver entry point, so the library does not link libcuda).
+// Host-side helpers of the launchers: encoding of TMA tensor maps
+// (cuTensorMapEncodeTiled through the runtime's driver entry point, so the
+// library does not link libcuda) and the cached dynamic shared-memory limits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
+#include <vector>
 
 #include "kernels.h"
 
@@ -32,6 +34,35 @@ int encode_tmap_bf16_4d(CUtensorMap* map, const void* base, const uint64_t dims[
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? 0 : (int)r;
+}
+
+namespace {
+struct SmemLimit {
+  int device;
+  const void* kernel;
+  int bytes;
+};
+std::mutex g_smem_mu;
+std::vector<SmemLimit> g_smem;
+}  // namespace
+
+cudaError_t ensure_dynamic_smem(const void* kernel, int bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(g_smem_mu);
+  for (SmemLimit& x : g_smem) {
+    if (x.device == dev && x.kernel == kernel) {
+      if (x.bytes >= bytes) return cudaSuccess;
+      if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess)
+        return e;
+      x.bytes = bytes;
+      return cudaSuccess;
+    }
+  }
+  if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess) return e;
+  g_smem.push_back({dev, kernel, bytes});
+  return cudaSuccess;
 }
 
 }  // namespace skv
