@@ -23,13 +23,9 @@
 // split across CTAs to fill the SMs; each split writes (O/l, log2-sum-exp)
 // partials that attn_combine merges, or out and lse directly when unsplit.
 //
-// Warp roles (640 threads): warp 0 TMA producer, warp 1 TMEM allocator + MMA
-// issuer, warps 4..11 softmax of tile A, warps 12..19 softmax of tile B.  Each
-// tile's rows are shared by two warpgroups that take 64 of the 128 key columns
-// each (warp w reads TMEM lanes 32*(w%4) .. +31, so each warpgroup covers all
-// 128 rows); the halves swap their row maxima through shared memory at a
-// named barrier, so a tile's softmax takes half as long on the critical chain
-// S(j) -> P(j) -> P.V(j) -> S(j+1).
+// Warp roles (384 threads): warp 0 TMA producer, warp 1 TMEM allocator + MMA
+// issuer, warps 4..7 softmax of tile A, warps 8..11 softmax of tile B (warp w
+// reads TMEM lanes 32*(w%4) .. +31, so each group covers all 128 rows).
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_common.cuh"
@@ -41,20 +37,14 @@ namespace {
 using namespace tc;
 
 constexpr int kSlots = 4;        // K/V ring slots (each one 128-key tile)
-// 20 warps: warpgroup 0 = TMA producer, MMA issuer and two idle warps; warps
-// 4..19 softmax.  Registers: launched at 96 per thread (640 x 96 = 61440);
-// warpgroup 0 drops to 64 and the four softmax warpgroups rise to 104:
-// 128 x 64 + 512 x 104 = 61440.
-constexpr int kSoftmaxWarp0 = 4;
-constexpr int kThreads = 32 * (kSoftmaxWarp0 + 16);
-constexpr int kRegsLaunch = 96;
-constexpr int kRegsLow = 64;
-constexpr int kRegsHigh = 104;
-static_assert(128 * kRegsLow + 512 * kRegsHigh <= kThreads * kRegsLaunch, "register split exceeds the launch");
+constexpr int kThreads = 384;
+// registers: launched at 168 per thread (384 x 168 = 64512); warpgroup 0
+// (producer, MMA issuer, two idle warps) drops to 72 and the two softmax
+// warpgroups rise to 216: 128 x 72 + 256 x 216 = 64512.
+constexpr int kRegsLow = 72;
+constexpr int kRegsHigh = 216;
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * 168, "register split exceeds the launch");
 constexpr float kRescaleLog2 = 8.0f;
-// Every kFmaExpEvery-th pair of P's exponentials runs on the FMA pipe
-// (exp2_fma) instead of MUFU, which otherwise issues all of them (0: none).
-constexpr int kFmaExpEvery = 0;
 
 template <int D>
 struct AttnSmem {
@@ -68,11 +58,7 @@ struct AttnSmem {
   static constexpr int kNumBars = 1 + 2 * kSlots + 6 + 1;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
-  // exchange of the two column halves' row maxima [parity][tile][half][row]
-  // and, at the end, of their row sums [tile][half][row]
-  static constexpr int kXmax = (kAbort + 4 + 15) & ~15;
-  static constexpr int kXl = kXmax + 2 * 2 * 2 * 128 * 4;
-  static constexpr int kBytes = kXl + 2 * 2 * 128 * 4;
+  static constexpr int kBytes = kAbort + 4;
   // at least 116 KB so that a second CTA (which would also need all 512 TMEM
   // columns) never shares the SM
   static constexpr int kAlloc = kBytes + 1024 > 116 * 1024 ? kBytes + 1024 : 116 * 1024;
@@ -158,7 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(bar_sfull(x), 1);
-      mbar_init(bar_pfull(x), 8);  // the eight warps of the tile's two softmax warpgroups
+      mbar_init(bar_pfull(x), 4);
       mbar_init(bar_odone(x), 1);
     }
     mbar_init(bar_done, 1);
@@ -179,7 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto col_s = [](int x) { return (uint32_t)(x * 128); };
   auto col_o = [](int x) { return (uint32_t)(256 + x * 128); };
 
-  if (warp < kSoftmaxWarp0) regs_dec<kRegsLow>();
+  if (warp < 4) regs_dec<kRegsLow>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -279,12 +265,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       drain_wait(bar_done, 0, a.err);
     }
     __syncwarp();
-  } else if (warp >= kSoftmaxWarp0) {
+  } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax
     regs_inc<kRegsHigh>();
-    const int wg = (warp - kSoftmaxWarp0) >> 2;  // softmax warpgroup 0..3
-    const int x = wg >> 1;           // 0: tile A, 1: tile B
-    const int half = wg & 1;         // key columns [64 * half, 64 * half + 64) of S
+    const int x = (warp - 4) >> 2;  // 0: tile A, 1: tile B
     const TileInfo ti = x == 0 ? tA : tB;
     const int nX = x == 0 ? nA : nB;
     const int quarter = warp & 3;
@@ -295,55 +279,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool row_exists = !a.stack || r < a.q_rows;
     const uint32_t t_s = tmem + ((uint32_t)(quarter * 32) << 16) + col_s(x);
     const uint32_t t_o = tmem + ((uint32_t)(quarter * 32) << 16) + col_o(x);
-    float* xmax = reinterpret_cast<float*>(smem + L::kXmax);
-    float* xl = reinterpret_cast<float*>(smem + L::kXl) + x * 256;
-    const int bar_id = 1 + x;  // named barrier of the tile's two warpgroups (256 threads)
     const float c = a.scale_log2;
     float m_used = -INFINITY, l = 0.f;
     bool ok = ti.valid;
     for (int j = 0; ok && j < nX; ++j) {
       // S_j is on the critical chain: spin (a suspending wait wakes later)
-      const bool got = warp_spin_wait(bar_sfull(x), j & 1, a.err, kErrWaitAcc, abort_flag, wait_lim);
-      uint32_t sv[64];
-      float mx = -INFINITY;
-      if (got) {
-        fence_after_sync();
-        const int k = kb + j;
-        const bool is_c = k < a.nC;
-        const int base = is_c ? k * 128 : (k - a.nC) * 128;
-        // visible columns of this row form a prefix [0, vis) of the tile
-        int vis = is_c ? a.m - base : (a.causal ? min(a.T, i + 1) : a.T) - base;
-        vis = max(0, min(64, max(0, min(128, vis)) - 64 * half));
-        const bool masked = __any_sync(0xffffffffu, vis < 64);
-        tmem_ld32(t_s + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(t_s + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        tmem_ld_wait();
-        if (masked) {
+      if (!(ok = warp_spin_wait(bar_sfull(x), j & 1, a.err, kErrWaitAcc, abort_flag, wait_lim))) break;
+      fence_after_sync();
+      const int k = kb + j;
+      const bool is_c = k < a.nC;
+      const int base = is_c ? k * 128 : (k - a.nC) * 128;
+      // visible columns of this row form a prefix [0, lim)
+      int lim = is_c ? a.m - base : (a.causal ? min(a.T, i + 1) : a.T) - base;
+      lim = max(0, min(128, lim));
+      const bool masked = __any_sync(0xffffffffu, lim < 128);
+      // the whole 128-column row of S in one batch of TMEM loads
+      uint32_t sv[128];
+      tmem_ld32(t_s + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+      tmem_ld32(t_s + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
+      tmem_ld32(t_s + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+      tmem_ld_wait();
+      if (masked) {
 #pragma unroll
-          for (int jj = 0; jj < 64; ++jj)
-            if (jj >= vis) sv[jj] = __float_as_uint(-INFINITY);
-        }
-        // max of this half of the row's raw logits (c > 0): four chains
-        float m4[4];
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          m4[q4] = __uint_as_float(sv[16 * q4]);
-#pragma unroll
-          for (int jj = 1; jj < 15; jj += 2)
-            m4[q4] = max3f(m4[q4], __uint_as_float(sv[16 * q4 + jj]), __uint_as_float(sv[16 * q4 + jj + 1]));
-          m4[q4] = fmaxf(m4[q4], __uint_as_float(sv[16 * q4 + 15]));
-        }
-        mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-        xmax[(((j & 1) * 2 + x) * 2 + half) * 128 + r] = mx;
+        for (int jj = 0; jj < 128; ++jj)
+          if (jj >= lim) sv[jj] = __float_as_uint(-INFINITY);
       }
-      // every warp of the tile's two warpgroups reaches this barrier once per
-      // tile, also when its wait gave up, so that all of them leave together
-      if (named_bar_red_or(bar_id, 256, !got)) {
-        ok = false;
-        break;
+      // row max of the raw logits (c > 0): eight independent chains
+      float m8[8];
+#pragma unroll
+      for (int q8 = 0; q8 < 8; ++q8) {
+        m8[q8] = __uint_as_float(sv[16 * q8]);
+#pragma unroll
+        for (int jj = 1; jj < 15; jj += 2)
+          m8[q8] = max3f(m8[q8], __uint_as_float(sv[16 * q8 + jj]), __uint_as_float(sv[16 * q8 + jj + 1]));
+        m8[q8] = fmaxf(m8[q8], __uint_as_float(sv[16 * q8 + 15]));
       }
-      // both halves have read their S columns: P may now overwrite them
-      mx = fmaxf(mx, xmax[(((j & 1) * 2 + x) * 2 + (half ^ 1)) * 128 + r]);
+      const float mx = fmaxf(fmaxf(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5])), fmaxf(m8[6], m8[7]));
       float m_new = fmaxf(m_used, mx * c);
       if (m_new == -INFINITY) m_new = 0.f;  // nothing visible yet in this row
       if (j == 0) {
@@ -351,43 +323,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         const bool need = m_new > m_used + kRescaleLog2;
         if (__any_sync(0xffffffffu, need)) {
-          // O holds P.V of earlier tiles, complete: S_j was issued after them.
-          // Each half rescales its half of O's columns.
+          // O holds P.V of earlier tiles, complete: S_j was issued after them
           const float f = need ? ex2_approx(m_used - m_new) : 1.f;
 #pragma unroll
           for (int c0 = 0; c0 < D / 32; ++c0) {
-            uint32_t v[16];
-            const uint32_t to = t_o + half * (D / 2) + c0 * 16;
-            tmem_ld16(to, v);
+            uint32_t v[32];
+            tmem_ld32(t_o + c0 * 32, v);
             tmem_ld_wait();
 #pragma unroll
-            for (int jj = 0; jj < 16; ++jj) v[jj] = __float_as_uint(__uint_as_float(v[jj]) * f);
-            tmem_st16(to, v);
+            for (int jj = 0; jj < 32; ++jj) v[jj] = __float_as_uint(__uint_as_float(v[jj]) * f);
+            tmem_st32(t_o + c0 * 32, v);
           }
           tmem_st_wait();
           l *= f;
           if (need) m_used = m_new;
         }
       }
-      // P = exp2(S*c - m_used) of this half's 64 columns (masked entries hold
-      // -inf -> 0), as bf16 pairs into TMEM columns [32*half, 32*half + 32)
+      // P = exp2(S*c - m_used) (masked entries hold -inf -> 0), as bf16 into
+      // the first 64 columns of the same TMEM region
       float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
-      for (int c0 = 0; c0 < 2; ++c0) {
+      for (int c0 = 0; c0 < 4; ++c0) {
         uint32_t pk[16];
 #pragma unroll
         for (int jj = 0; jj < 16; ++jj) {
-          const float x0 = fmaf(__uint_as_float(sv[c0 * 32 + 2 * jj]), c, -m_used);
-          const float x1 = fmaf(__uint_as_float(sv[c0 * 32 + 2 * jj + 1]), c, -m_used);
-          const bool on_fma = kFmaExpEvery > 0 && jj % (kFmaExpEvery > 0 ? kFmaExpEvery : 1) == 0;
-          // masked logits are -inf: exp2_fma would return a tiny value, not 0
-          const float p0 = on_fma ? (x0 == -INFINITY ? 0.f : exp2_fma(x0)) : ex2_approx(x0);
-          const float p1 = on_fma ? (x1 == -INFINITY ? 0.f : exp2_fma(x1)) : ex2_approx(x1);
+          const float p0 = ex2_approx(fmaf(__uint_as_float(sv[c0 * 32 + 2 * jj]), c, -m_used));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(sv[c0 * 32 + 2 * jj + 1]), c, -m_used));
           ls0 += p0;
           ls1 += p1;
           pk[jj] = pack_bf16x2(p0, p1);
         }
-        tmem_st16(t_s + 32 * half + c0 * 16, pk);
+        tmem_st16(t_s + c0 * 16, pk);
       }
       tmem_st_wait();
       l += ls0 + ls1;
@@ -395,24 +361,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_pfull(x));
     }
-    // ---- epilogue: the row sum of both halves, then O / l (each half writes
-    // its half of O's columns) and the row's log2-sum-exp
-    xl[half * 128 + r] = l;
-    named_bar_sync(bar_id, 256);  // every warp of the pair left the loop together
-    l += xl[(half ^ 1) * 128 + r];
+    // ---- epilogue: O / l and the row's log2-sum-exp
     if (ok && nX > 0) ok = warp_wait(bar_odone(x), 0, a.err, kErrWaitAcc, abort_flag, wait_lim);
     if (ok && ti.valid && !*abort_flag) {
       fence_after_sync();
       const bool row_ok = row_exists && i < a.T;
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const float lse2 = l > 0.f ? m_used + __log2f(l) : -INFINITY;
-      constexpr int kC = D / 64;  // 32-column chunks of O per half
       if (a.n_split == 1) {
         __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + s * a.out_s + (long long)i * a.out_row +
                               (long long)h * D;
 #pragma unroll
-        for (int cc = 0; cc < kC; ++cc) {
-          const int c0 = half * kC + cc;
+        for (int c0 = 0; c0 < D / 32; ++c0) {
           uint32_t v[32];
           tmem_ld32(t_o + c0 * 32, v);
           tmem_ld_wait();
@@ -426,12 +386,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int q4 = 0; q4 < 4; ++q4) dst[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
           }
         }
-        if (row_ok && a.lse && half == 0) a.lse[s * a.lse_s + (long long)h * a.T + i] = lse2 * kLn2;
+        if (row_ok && a.lse) a.lse[s * a.lse_s + (long long)h * a.T + i] = lse2 * kLn2;
       } else {
         const long long prow = ((long long)(s * a.Hq + h) * a.n_split + sp) * a.T + i;
 #pragma unroll
-        for (int cc = 0; cc < kC; ++cc) {
-          const int c0 = half * kC + cc;
+        for (int c0 = 0; c0 < D / 32; ++c0) {
           uint32_t v[32];
           if (nX > 0) {
             tmem_ld32(t_o + c0 * 32, v);
@@ -461,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (row_ok && half == 0) a.ml_part[prow] = nX > 0 ? lse2 : -INFINITY;
+        if (row_ok) a.ml_part[prow] = nX > 0 ? lse2 : -INFINITY;
       }
     }
   }

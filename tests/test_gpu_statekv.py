@@ -466,7 +466,8 @@ def _decode_case(wl, n_frames, n_text, dtype, device_frames=False, n_streams=1):
             args = [(torch.stack([f[i] for f in fr]) if n_streams > 1 else fr[0][i]).to(dev) for i in range(4)]
             h.prefill_frame(0, *args)
     # text tokens: the recipe's next frame, first n_text tokens
-    wl_txt = Syn.workload(wl.name, T=n_text, dist="iid", n_sinks=0, drift=0)
+    wl_txt = Syn.workload(wl.name, Hq=wl.Hq, Hkv=wl.Hkv, d=wl.d, dtype=dtype, T=n_text, dist="iid", n_sinks=0,
+                          drift=0)
     txt = [Syn.gen_frame(wl_txt, n_frames, stream=s) for s in range(n_streams)]
     q = torch.stack([t[0] for t in txt]) if n_streams > 1 else txt[0][0]
     k = torch.stack([t[1] for t in txt]) if n_streams > 1 else txt[0][1]
