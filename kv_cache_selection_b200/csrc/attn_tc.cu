@@ -54,8 +54,8 @@ struct AttnSmem {
   static constexpr int kQ = 0;                             // Q tiles A, B
   static constexpr int kKV = 2 * kTileBytes;               // ring
   static constexpr int kBar = kKV + kSlots * kTileBytes;
-  // q_full, kv_full[kSlots], kv_empty[kSlots], s_full[2], p_full[2], o_done[2], done
-  static constexpr int kNumBars = 1 + 2 * kSlots + 6 + 1;
+  // q_full, kv_full[kSlots], kv_empty[kSlots], s_full[2], p_full[2], o_done[2], done, pv_done
+  static constexpr int kNumBars = 1 + 2 * kSlots + 6 + 1 + 1;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4;
@@ -126,6 +126,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar_pfull = [&](int x) { return sb + L::kBar + 8u * (3 + 2 * kSlots + x); };
   auto bar_odone = [&](int x) { return sb + L::kBar + 8u * (5 + 2 * kSlots + x); };
   const uint32_t bar_done = sb + L::kBar + 8u * (7 + 2 * kSlots);
+  const uint32_t bar_pvdone = sb + L::kBar + 8u * (8 + 2 * kSlots);
+  // With no keys for tile B in this CTA (a lone query tile: decode, or the
+  // last tile of an odd count), tile A double-buffers S in the TMEM columns of
+  // S_B: S(j+1) is computed while the softmax of tile j runs.
+  const bool dbuf = nB == 0;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
   const unsigned long long wait_lim = a.wait_ns ? a.wait_ns : kWaitLimitNs;  // pipeline-wait limit
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
@@ -148,6 +153,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_odone(x), 1);
     }
     mbar_init(bar_done, 1);
+    mbar_init(bar_pvdone, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -234,6 +240,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j == nX[x] - 1) mma_commit(bar_odone(x));
       };
       bool ok = mbar_wait(bar_q, 0, a.err, kErrWaitLoad, abort_flag, wait_lim) && wait_slot(0);
+      if (dbuf) {
+        // S of tile j goes to buffer j & 1 (the S columns of tile A or B); the
+        // softmax of tile j overlaps S(j+1).  The tensor pipe runs MMAs in
+        // issue order, so S(j+1) overwrites P(j-1) only after P.V(j-1) read it.
+        auto issue_s_buf = [&](int buf, int j) {  // S_buf = Q_A K_j^T
+          const uint64_t dk = dk0 + slot16(2 * j);
+          const uint32_t d_tmem = tmem + col_s(buf);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = (uint64_t)(((kk >> 2) * L::kAtomBytes + (kk & 3) * 32) >> 4);
+            mma_ss(d_tmem, dq0 + off, dk + off, id_s, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar_sfull(buf));
+        };
+        if (ok) {
+          fence_after_sync();
+          issue_s_buf(0, 0);
+          mma_commit(bar_kvempty(0));
+        }
+        for (int j = 0; ok && j < nA; ++j) {
+          const bool next_k = j + 1 < nA;
+          if (next_k) {
+            if (!(ok = wait_slot(2 * (j + 1)))) break;  // K_{j+1}
+            issue_s_buf((j + 1) & 1, j + 1);
+          }
+          if (!(ok = wait_slot(2 * j + 1))) break;  // V_j
+          if (!(ok = mbar_wait(bar_pfull(j & 1), (j >> 1) & 1, a.err, kErrWaitP, abort_flag, wait_lim))) break;
+          fence_after_sync();
+          const uint64_t dv = dv0 + slot16(2 * j + 1);
+          const uint32_t a_tmem = tmem + col_s(j & 1);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + col_o(0), a_tmem + kk * 8, dv + (uint64_t)((kk * 2048) >> 4), id_o,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar_pvdone);
+          if (j == nA - 1) mma_commit(bar_odone(0));
+          mma_commit(bar_kvempty((2 * j + 1) % kSlots));                // V_j
+          if (next_k) mma_commit(bar_kvempty((2 * (j + 1)) % kSlots));  // K_{j+1}
+        }
+        ok = false;  // the paired loop below is for two query tiles
+      }
       if (ok) {
         fence_after_sync();
         if (nA > 0) issue_s(0, 0);
@@ -277,14 +324,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int i = a.stack ? ti.i0 + r / a.stack : ti.i0 + r;
     const int h = a.stack ? ti.h + r % a.stack : ti.h;
     const bool row_exists = !a.stack || r < a.q_rows;
-    const uint32_t t_s = tmem + ((uint32_t)(quarter * 32) << 16) + col_s(x);
-    const uint32_t t_o = tmem + ((uint32_t)(quarter * 32) << 16) + col_o(x);
+    const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t t_o = t_lane + col_o(x);
     const float c = a.scale_log2;
     float m_used = -INFINITY, l = 0.f;
     bool ok = ti.valid;
     for (int j = 0; ok && j < nX; ++j) {
+      // S of tile j: in buffer x, or in buffer j & 1 when tile A double-buffers
+      const int sbuf = dbuf ? (j & 1) : x;
+      const uint32_t sphase = dbuf ? ((j >> 1) & 1) : (j & 1);
+      const uint32_t t_s = t_lane + col_s(sbuf);
       // S_j is on the critical chain: spin (a suspending wait wakes later)
-      if (!(ok = warp_spin_wait(bar_sfull(x), j & 1, a.err, kErrWaitAcc, abort_flag, wait_lim))) break;
+      if (!(ok = warp_spin_wait(bar_sfull(sbuf), sphase, a.err, kErrWaitAcc, abort_flag, wait_lim))) break;
       fence_after_sync();
       const int k = kb + j;
       const bool is_c = k < a.nC;
@@ -323,7 +374,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         const bool need = m_new > m_used + kRescaleLog2;
         if (__any_sync(0xffffffffu, need)) {
-          // O holds P.V of earlier tiles, complete: S_j was issued after them
+          // O must hold P.V of every earlier tile: S_j was issued after them,
+          // except with double-buffered S, where P.V(j-1) may still run
+          if (dbuf && !(ok = warp_wait(bar_pvdone, (j - 1) & 1, a.err, kErrWaitAcc, abort_flag, wait_lim))) break;
+          fence_after_sync();
           const float f = need ? ex2_approx(m_used - m_new) : 1.f;
 #pragma unroll
           for (int c0 = 0; c0 < D / 32; ++c0) {
@@ -359,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       l += ls0 + ls1;
       fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_pfull(x));
+      if (lane == 0) mbar_arrive(bar_pfull(sbuf));
     }
     // ---- epilogue: O / l and the row's log2-sum-exp
     if (ok && nX > 0) ok = warp_wait(bar_odone(x), 0, a.err, kErrWaitAcc, abort_flag, wait_lim);
