@@ -62,28 +62,28 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* w
 // B-th largest value) is found by histogram refinement: the values still in
 // play span [umin, umax]; a 4096-bin histogram over that span (bin width
 // 2^shift) locates the bin holding the B-th largest; the bin becomes the new
-// span.  As soon as that bin is one value wide (tau found) or holds at most
-// kBrute candidates, the refinement stops and those candidates are ranked
+// span.  As soon as that bin is one value wide (tau found) or holds at most 32
+// candidates, the refinement stops and one warp ranks those candidates
 // exactly by (value desc, pool index asc).  The result is (tau, need_eq): keep
 // every candidate above tau and the first need_eq candidates equal to tau in
 // pool order, which is position order, so ties go to the lower position.
 constexpr int kBins = 4096;
-constexpr int kBrute = 256;
+static_assert(kBins == 4 * kSelThreads, "each thread clears and scans four bins");
 
 struct SelShared {
   alignas(16) uint32_t hist[kBins];
   uint32_t warp_a[kSelWarps];
   uint32_t warp_b[kSelWarps];
-  uint32_t list_j[kBrute];
-  uint32_t list_u[kBrute];
+  uint32_t list_j[32];
+  uint32_t list_u[32];
   uint32_t list_n;
   uint32_t sel_bin, sel_above;
+  uint32_t vmin, vmax, total;
   uint32_t tau, need_eq;
 };
 
 __device__ __forceinline__ uint32_t warp_min_u32(uint32_t v) { return __reduce_min_sync(0xffffffffu, v); }
 __device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) { return __reduce_max_sync(0xffffffffu, v); }
-__device__ __forceinline__ uint32_t warp_add_u32(uint32_t v) { return __reduce_add_sync(0xffffffffu, v); }
 
 __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) {
   extern __shared__ uint32_t su[];  // [L] value bits
@@ -167,14 +167,15 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
   __syncthreads();
   if (a.B <= 0) return;  // nothing is kept (block-uniform)
 
-  // 2. threshold
+  // 2. threshold.  Shared memory serves one warp-wide access per clock, so
+  //    block-wide results are reduced by one warp and read once per thread.
   const bool keep_all = L <= a.B;
   uint32_t tau = 0, need_eq = 0;
   if (!keep_all) {
     uint32_t lo = 0, hi = 0xffffffffu;  // span of the values still in play (inclusive)
     uint32_t need = (uint32_t)a.B;      // how many of them are kept
-    for (int level = 0;; ++level) {
-      // exact span of the values in play
+    for (;;) {
+      // exact span of the values in play; the histogram is cleared meanwhile
       uint32_t vmin = 0xffffffffu, vmax = 0u;
       for (int j = threadIdx.x; j < L; j += kSelThreads) {
         const uint32_t u = su[j];
@@ -183,7 +184,7 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
           vmax = max(vmax, u);
         }
       }
-      for (int b = threadIdx.x; b < kBins; b += kSelThreads) sh.hist[b] = 0u;
+      reinterpret_cast<uint4*>(sh.hist)[threadIdx.x] = make_uint4(0u, 0u, 0u, 0u);
       vmin = warp_min_u32(vmin);
       vmax = warp_max_u32(vmax);
       if (lane == 0) {
@@ -191,13 +192,16 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
         sh.warp_b[warp] = vmax;
       }
       __syncthreads();
-      vmin = 0xffffffffu;
-      vmax = 0u;
-#pragma unroll 8
-      for (int w = 0; w < kSelWarps; ++w) {
-        vmin = min(vmin, sh.warp_a[w]);
-        vmax = max(vmax, sh.warp_b[w]);
+      if (warp == 0) {
+        const uint32_t m0 = warp_min_u32(sh.warp_a[lane]), m1 = warp_max_u32(sh.warp_b[lane]);
+        if (lane == 0) {
+          sh.vmin = m0;
+          sh.vmax = m1;
+        }
       }
+      __syncthreads();
+      vmin = sh.vmin;
+      vmax = sh.vmax;
       if (vmin == vmax) {  // every value in play is equal: it is tau
         tau = vmin;
         need_eq = need;
@@ -205,26 +209,17 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
       }
       const uint32_t span = vmax - vmin;
       const int shift = max(0, 32 - __clz(span) - 12);  // (span >> shift) < kBins
-      // histogram of the values in play (warp-aggregated shared atomics)
-      for (int j0 = 0; j0 < L; j0 += kSelThreads) {
-        const int j = j0 + threadIdx.x;
-        bool in = false;
-        uint32_t bin = 0;
-        if (j < L) {
-          const uint32_t u = su[j];
-          in = u >= vmin && u <= vmax;
-          bin = (u - vmin) >> shift;
-        }
-        const uint32_t act = __ballot_sync(0xffffffffu, in);
-        if (in) {
-          const uint32_t peers = __match_any_sync(act, bin);
-          if (lane == __ffs(peers) - 1) atomicAdd(&sh.hist[bin], __popc(peers));
-        }
+      // histogram of the values in play (shared atomics; lanes of a warp that
+      // hit one bin are serialised by the hardware)
+      for (int j = threadIdx.x; j < L; j += kSelThreads) {
+        const uint32_t u = su[j];
+        if (u >= vmin && u <= vmax) atomicAdd(&sh.hist[(u - vmin) >> shift], 1u);
       }
       __syncthreads();
-      // thread t owns bins [4t, 4t + 4); count of values in bins >= b is the
-      // total minus the exclusive prefix; the bin where it first reaches
-      // `need` from the top holds the need-th largest
+      // thread t owns bins [4t, 4t + 4): a block prefix sum (warp shuffles, then
+      // warp 0 over the 32 warp totals) gives the values in bins below 4t; the
+      // bin where the count from the top first reaches `need` holds the need-th
+      // largest
       const uint4 h4 = reinterpret_cast<const uint4*>(sh.hist)[threadIdx.x];
       const uint32_t mine = h4.x + h4.y + h4.z + h4.w;
       uint32_t incl = mine;
@@ -235,21 +230,27 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
       }
       if (lane == 31) sh.warp_a[warp] = incl;
       __syncthreads();
-      uint32_t before = 0, total = 0;
-#pragma unroll 8
-      for (int w = 0; w < kSelWarps; ++w) {
-        const uint32_t x = sh.warp_a[w];
-        before += w < warp ? x : 0u;
-        total += x;
+      if (warp == 0) {
+        const uint32_t w = sh.warp_a[lane];
+        uint32_t wi = w;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const uint32_t n = __shfl_up_sync(0xffffffffu, wi, off);
+          if (lane >= off) wi += n;
+        }
+        sh.warp_b[lane] = wi - w;  // values in the bins of lower warps
+        if (lane == 31) sh.total = wi;
       }
-      before += incl - mine;  // values in bins below 4t
+      if (threadIdx.x == 0) sh.list_n = 0u;
+      __syncthreads();
+      const uint32_t total = sh.total;
       {
         const uint32_t hh[4] = {h4.x, h4.y, h4.z, h4.w};
-        uint32_t below = before;
+        uint32_t below = sh.warp_b[warp] + incl - mine;  // values in bins below 4t
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const uint32_t ge = total - below;       // values in bins >= 4t + e
-          const uint32_t gt = ge - hh[e];          // values in bins > 4t + e
+          const uint32_t ge = total - below;  // values in bins >= 4t + e
+          const uint32_t gt = ge - hh[e];     // values in bins > 4t + e
           if (ge >= need && gt < need) {
             sh.sel_bin = 4 * threadIdx.x + e;
             sh.sel_above = gt;
@@ -257,9 +258,9 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
           below += hh[e];
         }
       }
-      if (threadIdx.x == 0) sh.list_n = 0u;
       __syncthreads();
       const uint32_t b = sh.sel_bin;
+      const uint32_t in_bin = sh.hist[b];
       need -= sh.sel_above;
       lo = vmin + (b << shift);
       hi = shift == 0 ? lo : (uint32_t)min((unsigned long long)vmax, (unsigned long long)lo + (1ull << shift) - 1ull);
@@ -268,8 +269,10 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
         need_eq = need;
         break;
       }
-      if (sh.hist[b] <= (uint32_t)kBrute) {
-        // rank the bin's candidates exactly: order (value desc, pool index asc)
+      if (in_bin <= 32u) {
+        // rank the bin's candidates exactly in one warp: order (value desc,
+        // pool index asc); the need-th is tau, the kept ties are the
+        // candidates equal to it ranked up to it
         for (int j = threadIdx.x; j < L; j += kSelThreads) {
           const uint32_t u = su[j];
           if (u >= lo && u <= hi) {
@@ -279,41 +282,29 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
           }
         }
         __syncthreads();
-        const uint32_t n = sh.list_n;
-        if (threadIdx.x < n) {
-          const uint32_t uj = sh.list_u[threadIdx.x], jj = sh.list_j[threadIdx.x];
+        if (warp == 0) {
+          const uint32_t n = sh.list_n;
+          const bool have = (uint32_t)lane < n;
+          const uint32_t uj = have ? sh.list_u[lane] : 0u, jj = have ? sh.list_j[lane] : 0xffffffffu;
           uint32_t rank = 0;
           for (uint32_t k = 0; k < n; ++k) {
-            const uint32_t uk = sh.list_u[k];
-            rank += (uk > uj || (uk == uj && sh.list_j[k] < jj)) ? 1u : 0u;
+            const uint32_t uk = __shfl_sync(0xffffffffu, uj, k), jk = __shfl_sync(0xffffffffu, jj, k);
+            rank += (uk > uj || (uk == uj && jk < jj)) ? 1u : 0u;
           }
-          // the need-th of the bin in that order is tau; the kept ties are the
-          // candidates equal to it ranked before it, plus itself
-          if (rank == need - 1) sh.tau = uj;
+          const uint32_t tmask = __ballot_sync(0xffffffffu, have && rank == need - 1);
+          const uint32_t t = __shfl_sync(0xffffffffu, uj, __ffs(tmask) - 1);
+          const uint32_t eq = __popc(__ballot_sync(0xffffffffu, have && uj == t && rank < need));
+          if (lane == 0) {
+            sh.tau = t;
+            sh.need_eq = eq;
+          }
         }
         __syncthreads();
         tau = sh.tau;
-        uint32_t eq = 0;
-        if (threadIdx.x < n) {
-          const uint32_t uj = sh.list_u[threadIdx.x], jj = sh.list_j[threadIdx.x];
-          if (uj == tau) {
-            uint32_t rank = 0;
-            for (uint32_t k = 0; k < n; ++k) {
-              const uint32_t uk = sh.list_u[k];
-              rank += (uk > uj || (uk == uj && sh.list_j[k] < jj)) ? 1u : 0u;
-            }
-            eq = rank < need ? 1u : 0u;
-          }
-        }
-        eq = warp_add_u32(eq);
-        if (lane == 0) sh.warp_a[warp] = eq;
-        __syncthreads();
-        need_eq = 0;
-#pragma unroll 8
-        for (int w = 0; w < kSelWarps; ++w) need_eq += sh.warp_a[w];
+        need_eq = sh.need_eq;
         break;
       }
-      __syncthreads();  // the hist and sel_* reads above finish before the next level rewrites them
+      __syncthreads();  // the bin's count and sel_* are read before the next level rewrites them
     }
   }
 

@@ -66,15 +66,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Bounded wait for the completion of the phase with the given parity.  The
-// abort flag and the clock are checked every 64 polls only, so a waiting
-// thread takes few issue slots from the warps that share its scheduler.
+// abort flag and the clock are checked after the first failed poll and then
+// every 64 polls only, so a waiting thread takes few issue slots from the
+// warps that share its scheduler.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err, int code,
                                           volatile int* abort_flag, unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
+    if (it == 1 || (it & 63u) == 0) {
       if (*abort_flag) return false;
       if (globaltimer_ns() - t0 > limit_ns) {
         atomicCAS(err, 0, code);
@@ -281,12 +282,15 @@ __device__ __forceinline__ bool warp_spin_wait(uint32_t bar, uint32_t parity, in
   unsigned long long t0 = 0;
   for (uint32_t it = 0;; ++it) {
     if (__any_sync(0xffffffffu, mbar_test_wait(bar, parity))) return true;  // phases complete for good
-    if ((it & 63u) == 0) {
+    if (it == 0) {
+      if ((threadIdx.x & 31) == 0) t0 = globaltimer_ns();
+      continue;
+    }
+    // the clock and the abort flag: after the first failed poll, then every 64
+    if (it == 1 || (it & 63u) == 0) {
       int stop = 0;
       if ((threadIdx.x & 31) == 0) {
-        if (it == 0) {
-          t0 = globaltimer_ns();
-        } else if (*abort_flag) {
+        if (*abort_flag) {
           stop = 1;
         } else if (globaltimer_ns() - t0 > limit_ns) {
           atomicCAS(err, 0, code);
