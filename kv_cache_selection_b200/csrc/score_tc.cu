@@ -55,8 +55,9 @@ struct Smem {
   static constexpr int kNumBars = 1 + 2 * kStages + 8 + 1;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
-  static constexpr int kLse = (kAbort + 4 + 15) & ~15;    // [G][n_ic*128] row statistics follow
-  static constexpr int kAlloc = kLse + 1024;              // + room to align the base to 1024
+  static constexpr int kLse = (kAbort + 4 + 15) & ~15;    // [kGroups][2][128] row statistics
+  static constexpr int kBytes = kLse + kGroups * 2 * 128 * 4;
+  static constexpr int kAlloc = kBytes + 1024;            // + room to align the base to 1024
 };
 
 // Exponentials of 16 columns (query rows i0 .. i0+15) of one key's TMEM lane,
@@ -156,6 +157,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (is_c) tma_load_4d(sb + L::kK + at * L::kAtomBytes, &tm_kc, bar_k, at * 64, r0, g, s);
         else tma_load_4d(sb + L::kK + at * L::kAtomBytes, &tm_kf, bar_k, at * 64, g, r0, s);
       }
+      // the group's query rows: ask L2 for all of them now
+      for (int c = 0; c < n_chunks; ++c)
+        for (int at = 0; at < L::kAtoms; ++at)
+          tma_prefetch_l2_4d(&tm_q, at * 64, g * G + c / per_head, (ic_min + c % per_head) * 128, s);
       int issued = 0;
       for (int c = 0; c < n_chunks; ++c) {
         const int st = c % kStages;
@@ -204,58 +209,57 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int half = ew >> 2;             // group: takes chunks half, half + kGroups, ...
     const int row = quarter * 32 + lane;  // key row within the tile
     const int key = r0 + row;
-    // row statistics of the whole group in log2 units, negated, -inf past the
-    // frame: log2-sum-exp = max + log2(sum 2^(ml_u - max)) over the
-    // attention's key splits (or the stored lse when unsplit).  Loads of a
-    // thread's rows are issued before any is used.
-    const int tpad = n_ic * 128;
-    float* lse_all = reinterpret_cast<float*>(smem + L::kLse);
-    constexpr int kRowsPerThread = 4;
-    for (int e0 = threadIdx.x - 128; e0 < G * tpad; e0 += 32 * kEpiWarps * kRowsPerThread) {
-      float vals[kRowsPerThread][8];
+    // Row statistics in log2 units, negated, -inf past the frame: for each of
+    // its chunks a warpgroup loads the 128 rows' statistics (one row per
+    // thread: log2-sum-exp = max + log2(sum 2^(ml_u - max)) over the
+    // attention's key splits, or the stored lse when unsplit) into its own
+    // shared buffer; the loads for the next chunk are in flight while the
+    // current chunk is processed.
+    float* lse_wg = reinterpret_cast<float*>(smem + L::kLse) + half * 256;  // [2 slots][128 rows]
+    const int r_wg = threadIdx.x & 127;                                     // row of the chunk this thread loads
+    const int bar_wg = 3 + half;                                            // named barrier of the warpgroup
+    float mlv[8];
+    auto load_stats = [&](int c) {
+      const int hh = c / per_head;
+      const int i = (ic_min + c % per_head) * 128 + r_wg;
+      const bool valid = i < a.T;
+      const long long rowbase = (long long)(s * a.Hq + g * G + hh);
 #pragma unroll
-      for (int q = 0; q < kRowsPerThread; ++q) {
-        const int e = e0 + q * 32 * kEpiWarps;
-        const int hh = e / tpad, i = e % tpad;
-        const bool valid = e < G * tpad && i < a.T;
-        const long long rowbase = (long long)(s * a.Hq + g * G + hh);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          vals[q][u] = -INFINITY;
-          if (valid && a.n_split > 1 && u < a.n_split) vals[q][u] = a.ml_part[(rowbase * a.n_split + u) * a.T + i];
-        }
-        if (valid && a.n_split <= 1) vals[q][0] = a.lse[rowbase * a.T + i] * kLog2e;
+      for (int u = 0; u < 8; ++u) {
+        mlv[u] = -INFINITY;
+        if (valid && a.n_split > 1 && u < a.n_split) mlv[u] = __ldg(a.ml_part + (rowbase * a.n_split + u) * a.T + i);
       }
+      if (valid && a.n_split <= 1) mlv[0] = __ldg(a.lse + rowbase * a.T + i) * kLog2e;
+    };
+    auto publish_stats = [&](float* dst) {
+      float mx = mlv[0];
 #pragma unroll
-      for (int q = 0; q < kRowsPerThread; ++q) {
-        const int e = e0 + q * 32 * kEpiWarps;
-        if (e >= G * tpad) continue;
-        float mx = vals[q][0];
+      for (int u = 1; u < 8; ++u) mx = fmaxf(mx, mlv[u]);
+      float l2 = mx;
+      if (a.n_split > 1 && mx > -INFINITY) {
+        float ssum = 0.f;
 #pragma unroll
-        for (int u = 1; u < 8; ++u) mx = fmaxf(mx, vals[q][u]);
-        float l2 = mx;
-        if (a.n_split > 1 && mx > -INFINITY) {
-          float ssum = 0.f;
-#pragma unroll
-          for (int u = 0; u < 8; ++u) ssum += vals[q][u] == -INFINITY ? 0.f : ex2_approx(vals[q][u] - mx);
-          l2 = mx + __log2f(ssum);
-        }
-        // rows past the frame have no statistics: -inf makes their weight 0
-        lse_all[e] = mx == -INFINITY ? -INFINITY : -l2;
+        for (int u = 0; u < 8; ++u) ssum += mlv[u] == -INFINITY ? 0.f : ex2_approx(mlv[u] - mx);
+        l2 = mx + __log2f(ssum);
       }
-    }
-    named_bar_sync(2, 32 * kEpiWarps);
+      // rows past the frame have no statistics: -inf makes their weight 0
+      dst[r_wg] = mx == -INFINITY ? -INFINITY : -l2;
+    };
+    if (half < n_chunks) load_stats(half);
     float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
     bool ok = true;
-    for (int c = half; c < n_chunks; c += kGroups) {
+    for (int c = half, it = 0; c < n_chunks; c += kGroups, ++it) {
       const int buf = c & 3;
-      const int hh = c / per_head;
       const int i0 = (ic_min + c % per_head) * 128;
-      const float* lse2 = lse_all + hh * tpad + i0;
+      float* lse2 = lse_wg + (it & 1) * 128;
+      publish_stats(lse2);
+      if (c + kGroups < n_chunks) load_stats(c + kGroups);
       uint32_t got = 1;
       if (lane == 0) got = mbar_wait(bar_accfull(buf), (c >> 2) & 1, a.err, kErrWaitAcc, abort_flag, wait_lim) ? 1u : 0u;
       got = __shfl_sync(0xffffffffu, got, 0);
-      if (!got) {
+      // the warpgroup's four warps pass together (also when a wait gave up);
+      // the barrier also publishes the chunk's row statistics
+      if (named_bar_red_or(bar_wg, 128, got == 0)) {
         ok = false;
         break;
       }
@@ -318,15 +322,13 @@ cudaError_t launch_score_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kc, c
   if (n_tiles == 0) return cudaSuccess;
   dim3 grid(n_tiles, a.Hkv, a.S);
   cudaError_t e;
-  const int n_ic = (a.T + 127) / 128;
-  const int lse_bytes = (a.Hq / a.Hkv) * n_ic * 128 * 4;
   if (d == 128) {
-    const int smem = Smem<128>::kAlloc + lse_bytes;
+    const int smem = Smem<128>::kAlloc;
     if ((e = ensure_dynamic_smem(score_tc_kernel<128>, smem)))
       return e;
     return launch_kernel(score_tc_kernel<128>, grid, dim3(kThreads), smem, st, pdl, tm_q, tm_kc, tm_kf, a);
   } else {
-    const int smem = Smem<64>::kAlloc + lse_bytes;
+    const int smem = Smem<64>::kAlloc;
     if ((e = ensure_dynamic_smem(score_tc_kernel<64>, smem)))
       return e;
     return launch_kernel(score_tc_kernel<64>, grid, dim3(kThreads), smem, st, pdl, tm_q, tm_kc, tm_kf, a);

@@ -140,9 +140,6 @@ int check_shape(statekv_t h, int S, int Hq, int Hkv, int d, int T, int B, int ma
     return set_err(h, STATEKV_ERR_UNSUPPORTED, "pool B+T=%lld above 28672", (long long)B + T);
   if ((long long)max_frames * T > (1LL << 30))
     return set_err(h, STATEKV_ERR_UNSUPPORTED, "max_frames*T too large");
-  // bf16 score pass keeps the row statistics of one KV group in shared memory
-  if (dtype == STATEKV_BF16 && (Hq / Hkv) * ((T + 127) / 128) > 112)
-    return set_err(h, STATEKV_ERR_UNSUPPORTED, "bf16 path needs (Hq/Hkv)*ceil(T/128) <= 112");
   return STATEKV_OK;
 }
 
