@@ -184,21 +184,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_4d(sb + L::kQ + L::kTileBytes + at * L::kAtomBytes, &tm_q, bar_q, at * 64, tB.h, tB.i0, s);
         }
       }
-      // Ask L2 for the whole key range of this CTA now: the ring holds two key
-      // tiles, and without the prefetch each of its loads waits for HBM.
-      for (int k = kb; k < kb + n_load; ++k) {
-        const bool is_c = k < a.nC;
-        const int r0 = is_c ? k * 128 : (k - a.nC) * 128;
-        for (int at = 0; at < L::kAtoms; ++at) {
-          if (is_c) {
-            tma_prefetch_l2_4d(&tm_kc, at * 64, r0, g, s);
-            tma_prefetch_l2_4d(&tm_vc, at * 64, r0, g, s);
-          } else {
-            tma_prefetch_l2_4d(&tm_kf, at * 64, g, r0, s);
-            tma_prefetch_l2_4d(&tm_vf, at * 64, g, r0, s);
-          }
-        }
-      }
       int issued = 0;
       for (int idx = 0; idx < 2 * n_load; ++idx) {
         const int sl = idx % kSlots;

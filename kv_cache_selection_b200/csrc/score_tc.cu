@@ -157,10 +157,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (is_c) tma_load_4d(sb + L::kK + at * L::kAtomBytes, &tm_kc, bar_k, at * 64, r0, g, s);
         else tma_load_4d(sb + L::kK + at * L::kAtomBytes, &tm_kf, bar_k, at * 64, g, r0, s);
       }
-      // the group's query rows: ask L2 for all of them now
-      for (int c = 0; c < n_chunks; ++c)
-        for (int at = 0; at < L::kAtoms; ++at)
-          tma_prefetch_l2_4d(&tm_q, at * 64, g * G + c / per_head, (ic_min + c % per_head) * 128, s);
       int issued = 0;
       for (int c = 0; c < n_chunks; ++c) {
         const int st = c % kStages;
