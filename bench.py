@@ -362,7 +362,7 @@ def run_ours(args, wl):
         "roofline": roofline,
         "stages_us": per_stage,
         "stages_note": ("per-kernel CUDA events in a second pass of K steps (events serialise the kernels); "
-                        "the attention kernel merges its own key splits"),
+                        "attention includes the merge of its key splits, launched on its own in that pass"),
         "step_us_p50": round(statistics.median(ms_steps) * 1e3, 2),
         "step_us_p99": round(sorted(ms_steps)[int(0.99 * (len(ms_steps) - 1))] * 1e3, 2),
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),

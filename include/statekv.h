@@ -183,7 +183,7 @@ int statekv_get_step_stats(statekv_t h, const float** lse, const float** pool_sc
 /* Kernel stages of one step, for statekv_profile_read. */
 typedef enum {
   STATEKV_STAGE_ATTENTION = 0,         /* (a) attention main kernel            */
-  STATEKV_STAGE_ATTENTION_COMBINE = 1, /* not recorded: the attention kernel merges its own key splits */
+  STATEKV_STAGE_ATTENTION_COMBINE = 1, /* (a) merge of key-split partials      */
   STATEKV_STAGE_SCORE = 2,             /* (b) score pass                       */
   STATEKV_STAGE_SELECT = 3,            /* (c) top-B select                     */
   STATEKV_STAGE_GATHER = 4,            /* (d) gather into C_n + append to D    */
@@ -194,8 +194,10 @@ typedef enum {
 
 /* Per-stage device timing: when on, every later prefill_frame records a CUDA
  * event pair around each kernel on the call's stream (a few microseconds of
- * extra enqueue cost; leave off in production).  Turning it off drops
- * unread records. */
+ * extra enqueue cost; leave off in production), and the merge of the
+ * attention's key splits, which otherwise rides in the select launch, runs as
+ * its own launch so that its time is recorded under ATTENTION_COMBINE.
+ * Turning it off drops unread records. */
 int statekv_profile_enable(statekv_t h, int on);
 
 /* Accumulated device time and launch count per stage since the last read:

@@ -21,8 +21,7 @@
 // O and the row sum are rescaled only when a row's max grows by more than 2^8,
 // so P stays below 256 and the result is exact up to rounding.  Key tiles are
 // split across CTAs to fill the SMs; each split writes (O/l, log2-sum-exp)
-// partials, and the last split CTA of a tile pair to finish merges them into
-// out and lse (or out and lse are written directly when unsplit).
+// partials that attn_combine merges, or out and lse directly when unsplit.
 //
 // Warp roles (384 threads): warp 0 TMA producer, warp 1 TMEM allocator + MMA
 // issuer, warps 4..7 softmax of tile A, warps 8..11 softmax of tile B (warp w
@@ -59,8 +58,7 @@ struct AttnSmem {
   static constexpr int kNumBars = 1 + 2 * kSlots + 6 + 1 + 1;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
-  static constexpr int kLast = kAbort + 4;  // this CTA merges the tile pair's splits
-  static constexpr int kBytes = kLast + 4;
+  static constexpr int kBytes = kAbort + 4;
   // at least 116 KB so that a second CTA (which would also need all 512 TMEM
   // columns) never shares the SM
   static constexpr int kAlloc = kBytes + 1024 > 116 * 1024 ? kBytes + 1024 : 116 * 1024;
@@ -99,8 +97,7 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kc,
                    const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_kf,
-                   const __grid_constant__ CUtensorMap tm_vf, const __grid_constant__ CUtensorMap tm_o,
-                   AttnTcArgs a) {
+                   const __grid_constant__ CUtensorMap tm_vf, AttnTcArgs a) {
   using L = AttnSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -145,7 +142,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tm_vc);
     tma_prefetch_desc(&tm_kf);
     tma_prefetch_desc(&tm_vf);
-    if (a.o_tma) tma_prefetch_desc(&tm_o);
     mbar_init(bar_q, 1);
     for (int sl = 0; sl < kSlots; ++sl) {
       mbar_init(bar_kvfull(sl), 1);
@@ -421,61 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // ---- epilogue: O / l and the row's log2-sum-exp
     if (ok && nX > 0) ok = warp_wait(bar_odone(x), 0, a.err, kErrWaitAcc, abort_flag, wait_lim);
-    if (a.o_tma && ti.valid) {
-      // O/l as bf16 into this tile's query buffer (its S MMAs are complete),
-      // in the 128-byte-swizzled layout of the tensor map, then two TMA
-      // stores (one per 64-column atom) by one thread.  The tile's four warps
-      // pass the barrier together, also when one of their waits gave up.
-      const bool fine = ok && !*abort_flag;
-      uint8_t* stage = smem + L::kQ + x * L::kTileBytes;
-      const bool row_ok = row_exists && i < a.T;
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      const float lse2 = l > 0.f ? m_used + __log2f(l) : -INFINITY;
-      if (fine) {
-        fence_after_sync();
-#pragma unroll
-        for (int c0 = 0; c0 < D / 32; ++c0) {
-          uint32_t v[32];
-          if (nX > 0) {
-            tmem_ld32(t_o + c0 * 32, v);
-            tmem_ld_wait();
-          } else {
-#pragma unroll
-            for (int jj = 0; jj < 32; ++jj) v[jj] = 0u;
-          }
-          uint32_t pk[16];
-#pragma unroll
-          for (int jj = 0; jj < 16; ++jj)
-            pk[jj] = pack_bf16x2(__uint_as_float(v[2 * jj]) * inv, __uint_as_float(v[2 * jj + 1]) * inv);
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const int c16 = c0 * 4 + q4;  // 16-byte chunk of the row (8 columns)
-            uint8_t* dst = stage + (c16 >> 3) * L::kAtomBytes + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
-            *reinterpret_cast<uint4*>(dst) = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
-          }
-        }
-        fence_proxy_async_smem();
-      }
-      const bool bad = named_bar_red_or(1 + x, 128, !fine);
-      if (!bad) {
-        if (quarter == 0 && lane == 0) {
-          for (int at = 0; at < L::kAtoms; ++at) {
-            if (a.n_split == 1) tma_store_4d(&tm_o, smem_u32(stage + at * L::kAtomBytes), at * 64, ti.h, ti.i0, s);
-            else tma_store_4d(&tm_o, smem_u32(stage + at * L::kAtomBytes), at * 64, ti.i0, sp, s * a.Hq + ti.h);
-          }
-          bulk_commit();
-          bulk_wait_all();
-          fence_proxy_async_global();
-        }
-        if (row_ok) {
-          if (a.n_split == 1) {
-            if (a.lse) a.lse[s * a.lse_s + (long long)h * a.T + i] = lse2 * kLn2;
-          } else {
-            a.ml_part[((long long)(s * a.Hq + h) * a.n_split + sp) * a.T + i] = nX > 0 ? lse2 : -INFINITY;
-          }
-        }
-      }
-    } else if (ok && ti.valid && !*abort_flag) {
+    if (ok && ti.valid && !*abort_flag) {
       fence_after_sync();
       const bool row_ok = row_exists && i < a.T;
       const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -537,37 +479,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   fence_before_sync();
-  // the split partials written above are visible device-wide before this
-  // CTA's arrival is counted
-  __threadfence();
   __syncthreads();
   if (warp == 1) {
     fence_after_sync();
     tmem_dealloc(tmem, 512);
   }
-  // Merge of the key splits: the last split CTA of the tile pair to arrive
-  // merges the pair's rows (no CTA waits for another) and resets the counter
-  // for the next launch.
-  if (a.merge_count && a.n_split > 1 && !a.o_part32) {
-    volatile int* last = reinterpret_cast<volatile int*>(smem + L::kLast);
-    const int pair_unit = blockIdx.x / a.n_split;
-    if (threadIdx.x == 0) *last = atomicAdd(a.merge_count + pair_unit, 1) == a.n_split - 1;
-    __syncthreads();
-    if (*last) {
-      __threadfence();
-      constexpr int kChunks = D / 8;
-      for (int t = threadIdx.x; t < 2 * 128 * kChunks; t += kThreads) {
-        const int x = t / (128 * kChunks);
-        const TileInfo& ti = x == 0 ? tA : tB;
-        const int r = (t / kChunks) % 128;
-        const int i = ti.i0 + r;
-        if (ti.valid && i < a.T)
-          merge_row_chunk<D>(a.out, a.out_s, a.out_row, a.lse, a.lse_s, a.o_part, a.ml_part, a.Hq, a.T, a.n_split, s,
-                             ti.h, i, t % kChunks);
-      }
-      if (threadIdx.x == 0) a.merge_count[pair_unit] = 0;
-    }
-  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) attn_combine_kernel(MergeArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  merge_chunk<D>(a, blockIdx.x * blockDim.x + threadIdx.x);
 }
 
 // Merge of n_split float32 partials (O/l and log2-sum-exp per split): thread
@@ -635,8 +558,8 @@ int attn_tc_splits(int S, int Hq, int Hkv, int T, int m, int n_sm) {
 }
 
 cudaError_t launch_attn_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kc, const CUtensorMap& tm_vc,
-                           const CUtensorMap& tm_kf, const CUtensorMap& tm_vf, const CUtensorMap& tm_o,
-                           const AttnTcArgs& a, int d, cudaStream_t st, bool pdl) {
+                           const CUtensorMap& tm_kf, const CUtensorMap& tm_vf, const AttnTcArgs& a, int d,
+                           cudaStream_t st, bool pdl) {
   const int units = a.S * a.Hkv * a.n_pairs * a.n_split;
   cudaError_t e;
   if (d == 128) {
@@ -644,16 +567,40 @@ cudaError_t launch_attn_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kc, co
     if ((e = ensure_dynamic_smem(attn_tc_kernel<128>, smem)))
       return e;
     return launch_kernel(attn_tc_kernel<128>, dim3(units), dim3(kThreads), smem, st, pdl, tm_q, tm_kc, tm_vc,
-                         tm_kf, tm_vf, tm_o, a);
+                         tm_kf, tm_vf, a);
   } else {
     const int smem = AttnSmem<64>::kAlloc;
     if ((e = ensure_dynamic_smem(attn_tc_kernel<64>, smem)))
       return e;
     return launch_kernel(attn_tc_kernel<64>, dim3(units), dim3(kThreads), smem, st, pdl, tm_q, tm_kc, tm_vc,
-                         tm_kf, tm_vf, tm_o, a);
+                         tm_kf, tm_vf, a);
   }
   return cudaGetLastError();
 }
 
+MergeArgs merge_args(const AttnTcArgs& a, int d) {
+  MergeArgs m{};
+  m.out = a.out;
+  m.out_s = a.out_s;
+  m.out_row = a.out_row;
+  m.lse = a.lse;
+  m.lse_s = a.lse_s;
+  m.o_part = a.o_part;
+  m.ml_part = a.ml_part;
+  m.S = a.S;
+  m.Hq = a.Hq;
+  m.T = a.T;
+  m.n_split = a.n_split;
+  m.d = d;
+  return m;
+}
+
+cudaError_t launch_attn_combine(const AttnTcArgs& a, int d, cudaStream_t st, bool pdl) {
+  const MergeArgs m = merge_args(a, d);
+  const long long rows = (long long)a.S * a.Hq * a.T;
+  const int blocks = (int)((rows * (d / 8) + 255) / 256);
+  if (d == 128) return launch_kernel(attn_combine_kernel<128>, dim3(blocks), dim3(256), 0, st, pdl, m);
+  return launch_kernel(attn_combine_kernel<64>, dim3(blocks), dim3(256), 0, st, pdl, m);
+}
 
 }  // namespace skv

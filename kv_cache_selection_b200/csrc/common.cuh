@@ -77,7 +77,21 @@ struct ScoreArgs {
   float scale_log2;
 };
 
-// Top-B selection over the pool of one (stream, selection group).
+// Merge of the attention's key-split partials into out and lse.
+struct MergeArgs {
+  void* out;                     // out[s][i][h][dd] bf16
+  long long out_s;
+  int out_row;
+  float* lse;                    // [S][Hq][T] natural log, may be null
+  long long lse_s;
+  const __nv_bfloat16* o_part;   // [S][Hq][n_split][T][d] O/l per split
+  const float* ml_part;          // [S][Hq][n_split][T] log2-sum-exp
+  int S, Hq, T, n_split, d;
+};
+
+// Top-B selection over the pool of one (stream, selection group).  The same
+// launch carries extra blocks that merge the attention's key-split partials
+// (not on the path to C_n).
 struct SelectArgs {
   const float* part;      // part[s][g][j], j < m + T
   long long part_s;
@@ -88,7 +102,10 @@ struct SelectArgs {
   int32_t* idx;           // out [s][g][B] kept pool indices, ascending (row 0 in global mode)
   int Hkv, m, T, B, global;
   int recency;            // keep the B largest positions instead of the B largest scores
-  int n_sel_blocks;       // one block per (stream, selection group)
+  int n_sel_blocks;       // blocks [0, n_sel_blocks): one per (stream, selection group)
+  // key-split merge (n_mrg_blocks > 0 only for the bf16 attention with splits)
+  int n_mrg_blocks;
+  MergeArgs mrg;
 };
 
 // Gather of the kept rows into the next C buffer, plus the append of the

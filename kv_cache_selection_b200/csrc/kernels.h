@@ -89,22 +89,15 @@ struct AttnTcArgs {
   float scale_log2;
   int* err;
   unsigned long long wait_ns;  // pipeline-wait limit; 0 = the default
-  // bf16 partials (n_split > 1): one zero-initialised counter per (stream, KV
-  // group, tile pair); the last split CTA of a pair to finish merges the
-  // pair's rows into out and lse and resets the counter
-  int* merge_count;
-  // o_tma = 1: O is written with TMA stores through the map tm_o, staged in
-  // the query tile's shared memory (not for stacked tiles or float32
-  // partials): over out [S][T][Hq][d] as {d, Hq, T, S} when n_split == 1,
-  // over o_part as {d, T, n_split, S*Hq} otherwise, boxes of 64 x 128 rows
-  int o_tma;
 };
 int attn_tc_splits(int S, int Hq, int Hkv, int T, int m, int n_sm);
 cudaError_t launch_attn_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kc, const CUtensorMap& tm_vc,
-                           const CUtensorMap& tm_kf, const CUtensorMap& tm_vf, const CUtensorMap& tm_o,
-                           const AttnTcArgs& a, int d, cudaStream_t st, bool pdl = false);
+                           const CUtensorMap& tm_kf, const CUtensorMap& tm_vf, const AttnTcArgs& a, int d,
+                           cudaStream_t st, bool pdl = false);
+cudaError_t launch_attn_combine(const AttnTcArgs& a, int d, cudaStream_t st, bool pdl = false);
 // Merge of any number of float32 key-split partials (o_part32) into out and lse.
 cudaError_t launch_attn_merge_wide(const AttnTcArgs& a, int d, cudaStream_t st, bool pdl = false);
+MergeArgs merge_args(const AttnTcArgs& a, int d);
 
 // Message for statekv_last_error(NULL) (errors of calls without a handle).
 void set_free_error(const char* msg);

@@ -12,6 +12,7 @@
 // C_{n-1} is, and every frame position exceeds all earlier ones).
 #include "common.cuh"
 #include "kernels.h"
+#include "merge.cuh"
 
 namespace skv {
 namespace {
@@ -89,6 +90,13 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
   __shared__ SelShared sh;
   pdl_wait();
   pdl_trigger();
+  if ((int)blockIdx.x >= a.n_sel_blocks) {
+    // extra blocks: merge of the attention's key-split partials
+    const int t = (blockIdx.x - a.n_sel_blocks) * kSelThreads + threadIdx.x;
+    if (a.mrg.d == 128) merge_chunk<128>(a.mrg, t);
+    else merge_chunk<64>(a.mrg, t);
+    return;
+  }
   const int n_groups = a.global ? 1 : a.Hkv;
   const int grp = blockIdx.x % n_groups, s = blockIdx.x / n_groups;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -432,6 +440,12 @@ cudaError_t launch_select(const SelectArgs& a_in, int S, cudaStream_t st, bool p
   const int L = a.m + a.T;
   const int n_groups = a.global ? 1 : a.Hkv;
   a.n_sel_blocks = n_groups * S;
+  if (a.mrg.n_split > 1) {
+    const long long mrg_threads = (long long)a.mrg.S * a.mrg.Hq * a.mrg.T * (a.mrg.d / 8);
+    a.n_mrg_blocks = (int)((mrg_threads + kSelThreads - 1) / kSelThreads);
+  } else {
+    a.n_mrg_blocks = 0;
+  }
   const size_t smem = (size_t)L * sizeof(uint32_t);
   // the default 48 KB per block covers static and dynamic shared memory
   // together; the kernel's static arrays take ~19 KB, so opt in above 24 KB
@@ -439,7 +453,8 @@ cudaError_t launch_select(const SelectArgs& a_in, int S, cudaStream_t st, bool p
     cudaError_t e = ensure_dynamic_smem(select_topb_kernel, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  return launch_kernel(select_topb_kernel, dim3(a.n_sel_blocks), dim3(kSelThreads), smem, st, pdl, a);
+  return launch_kernel(select_topb_kernel, dim3(a.n_sel_blocks + a.n_mrg_blocks), dim3(kSelThreads), smem, st,
+                       pdl, a);
 }
 
 template <int VPR>

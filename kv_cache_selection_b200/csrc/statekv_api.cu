@@ -47,7 +47,6 @@ struct LayerState {
   __nv_bfloat16* o_part = nullptr;  // attention key-split partials (bf16 path)
   float* ml_part = nullptr;
   int pool_len = 0;             // pool size of the layer's last step
-  int* merge_count = nullptr;   // [S][Hkv][tile pairs] split counters of the attention
 };
 
 }  // namespace
@@ -165,11 +164,9 @@ int alloc_layer(statekv_t h, LayerState& L) {
       (rc = dev_alloc(h, (void**)&L.pool_score, S * h->Hkv * pool * 4)) ||
       (rc = dev_alloc(h, (void**)&L.idx, S * h->Hkv * std::max(h->B, 1) * 4)))
     return rc;
-  const size_t n_pairs = ((size_t)(h->Hq / h->Hkv) * ((h->T + 127) / 128) + 1) / 2;
   if (h->max_split > 1 &&
       ((rc = dev_alloc(h, (void**)&L.o_part, S * h->Hq * h->max_split * h->T * h->d * 2)) ||
-       (rc = dev_alloc(h, (void**)&L.ml_part, S * h->Hq * h->max_split * h->T * 4)) ||
-       (rc = dev_alloc(h, (void**)&L.merge_count, S * h->Hkv * n_pairs * 4))))
+       (rc = dev_alloc(h, (void**)&L.ml_part, S * h->Hq * h->max_split * h->T * 4))))
     return rc;
   L.ready = true;
   return STATEKV_OK;
@@ -248,23 +245,6 @@ int encode_step_maps(statekv_t h, const void* q, const void* kc, const void* k, 
   return STATEKV_OK;
 }
 
-// TMA map through which the attention stores O: over out [S][T][Hq][d] when
-// unsplit, else over the split partials [S*Hq][n_split][T][d].
-int encode_out_map(CUtensorMap* map, void* out, const __nv_bfloat16* o_part, int S, int Hq, int T, int d,
-                   int n_split) {
-  const uint64_t D = d;
-  const uint32_t box_out[4] = {64, 1, 128, 1};
-  const uint32_t box_part[4] = {64, 128, 1, 1};
-  if (n_split <= 1) {
-    const uint64_t dims[4] = {D, (uint64_t)Hq, (uint64_t)T, (uint64_t)S};
-    const uint64_t str[3] = {D * 2, (uint64_t)Hq * D * 2, (uint64_t)T * Hq * D * 2};
-    return skv::encode_tmap_bf16_4d(map, out, dims, str, box_out);
-  }
-  const uint64_t dims[4] = {D, (uint64_t)T, (uint64_t)n_split, (uint64_t)S * Hq};
-  const uint64_t str[3] = {D * 2, (uint64_t)T * D * 2, (uint64_t)n_split * T * D * 2};
-  return skv::encode_tmap_bf16_4d(map, o_part, dims, str, box_part);
-}
-
 int launch_err(statekv_t h, cudaError_t e, const char* what) {
   return set_err(h, STATEKV_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString(e));
 }
@@ -284,8 +264,7 @@ struct FcScratch {
   __nv_bfloat16* o = nullptr;
   float* ml = nullptr;
   int* err = nullptr;
-  int* count = nullptr;  // split counters of the attention's in-kernel merge (kept at zero)
-  size_t o_bytes = 0, ml_bytes = 0, count_bytes = 0;
+  size_t o_bytes = 0, ml_bytes = 0;
 };
 FcScratch g_fc[64];
 
@@ -342,22 +321,10 @@ int full_causal_tc(const void* q, const void* k, const void* v, int n_seq, int N
       }
       sc.ml_bytes = mb;
     }
-    const size_t cb = ta.n_split > 1 ? (size_t)n_seq * Hkv * ta.n_pairs * 4 : 16;
-    if (sc.count_bytes < cb) {
-      if (sc.count) cudaFree(sc.count);
-      sc.count = nullptr;
-      sc.count_bytes = 0;
-      if (cudaMalloc((void**)&sc.count, cb) != cudaSuccess || cudaMemset(sc.count, 0, cb) != cudaSuccess) {
-        cudaGetLastError();
-        return set_err(nullptr, STATEKV_ERR_OOM, "scratch allocation of %zu bytes failed", cb);
-      }
-      sc.count_bytes = cb;
-    }
     if (!sc.err) return set_err(nullptr, STATEKV_ERR_OOM, "error-word allocation failed");
     ta.o_part = sc.o;
     ta.ml_part = sc.ml;
     ta.err = sc.err;
-    ta.merge_count = sc.count;
   }
   // q [S][N][Hq][d] and k, v [S][N][Hkv][d]: the whole sequence is the "frame"
   const uint64_t D = d;
@@ -371,13 +338,11 @@ int full_causal_tc(const void* q, const void* k, const void* v, int n_seq, int N
   if ((r = skv::encode_tmap_bf16_4d(&tq, q, dq, sq, box)) || (r = skv::encode_tmap_bf16_4d(&tk, k, dk, sk, box)) ||
       (r = skv::encode_tmap_bf16_4d(&tv, v, dk, sk, box)))
     return set_err(nullptr, STATEKV_ERR_CUDA, "TMA tensor map encoding failed (CUresult %d)", r);
-  CUtensorMap to;
-  if ((r = encode_out_map(&to, out, ta.o_part, n_seq, Hq, N, d, ta.n_split)))
-    return set_err(nullptr, STATEKV_ERR_CUDA, "TMA tensor map encoding failed (CUresult %d)", r);
-  ta.o_tma = 1;
   // no compressed rows: the C maps are never read
-  if ((e = skv::launch_attn_tc(tq, tk, tv, tk, tv, to, ta, d, st)) != cudaSuccess)
+  if ((e = skv::launch_attn_tc(tq, tk, tv, tk, tv, ta, d, st)) != cudaSuccess)
     return set_err(nullptr, STATEKV_ERR_CUDA, "attention launch failed: %s", cudaGetErrorString(e));
+  if (ta.n_split > 1 && (e = skv::launch_attn_combine(ta, d, st)) != cudaSuccess)
+    return set_err(nullptr, STATEKV_ERR_CUDA, "attention combine launch failed: %s", cudaGetErrorString(e));
   return STATEKV_OK;
 }
 
@@ -482,6 +447,8 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
   aa.causal = h->mask == STATEKV_MASK_FRAME_CAUSAL;
   aa.scale_log2 = scale_log2;
   CUtensorMap tq, tkc, tkf, tvc, tvf;
+  skv::MergeArgs mrg{};  // key-split merge, run by the select launch (bf16 with splits)
+  int n_split = 1;
   if (h->dtype == STATEKV_BF16) {
     if ((rc = encode_step_maps(h, q, L->kc[cur], k, &tq, &tkc, &tkf, L->vc[cur], v, &tvc, &tvf))) return rc;
     skv::AttnTcArgs ta{};
@@ -508,17 +475,23 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
     ta.scale_log2 = scale_log2;
     ta.err = h->dev_err;
     ta.wait_ns = h->wait_ns;
-    ta.merge_count = L->merge_count;  // the attention merges its own key splits
-    CUtensorMap to;
-    int r;
-    if ((r = encode_out_map(&to, out, L->o_part, S, Hq, T, d, ta.n_split)))
-      return set_err(h, STATEKV_ERR_CUDA, "TMA tensor map encoding failed (CUresult %d)", r);
-    ta.o_tma = 1;
     {
       StageScope sc(h, st, STATEKV_STAGE_ATTENTION);
-      if ((e = skv::launch_attn_tc(tq, tkc, tvc, tkf, tvf, to, ta, d, st, true)) != cudaSuccess)
+      if ((e = skv::launch_attn_tc(tq, tkc, tvc, tkf, tvf, ta, d, st, true)) != cudaSuccess)
         return launch_err(h, e, "attention");
       sc.done();
+    }
+    n_split = ta.n_split;
+    if (n_split > 1) {
+      if (h->prof) {
+        // timed runs charge the merge of the key splits to the attention stage
+        // by launching it on its own; otherwise it rides in the select launch
+        StageScope sc(h, st, STATEKV_STAGE_ATTENTION_COMBINE);
+        if ((e = skv::launch_attn_combine(ta, d, st, true)) != cudaSuccess) return launch_err(h, e, "attention merge");
+        sc.done();
+      } else {
+        mrg = skv::merge_args(ta, d);
+      }
     }
   } else {
     StageScope sc(h, st, STATEKV_STAGE_ATTENTION);
@@ -554,7 +527,7 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
     ta.lse = L->lse;
     ta.lse_s = aa.lse_s;
     ta.ml_part = L->ml_part;
-    ta.n_split = 1;  // the attention wrote the merged lse
+    ta.n_split = n_split;
     ta.part = L->part;
     ta.part_s = sa.part_s;
     ta.part_g = pool;
@@ -593,6 +566,7 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
   se.B = B;
   se.global = h->select != STATEKV_SELECT_PER_KV_HEAD;  // recency keeps one set per layer too
   se.recency = h->select == STATEKV_SELECT_RECENCY;
+  se.mrg = mrg;
   {
     StageScope sc(h, st, STATEKV_STAGE_SELECT);
     if ((e = skv::launch_select(se, S, st, true)) != cudaSuccess) return launch_err(h, e, "select");
@@ -808,8 +782,7 @@ int statekv_decode(statekv_t h, int layer, const void* q, const void* k, const v
     return set_err(h, STATEKV_ERR_CUDA, "TMA tensor map encoding failed (CUresult %d)", r);
   {
     StageScope sc(h, st, STATEKV_STAGE_DECODE);
-    // stacked tiles store O thread by thread (o_tma = 0): the map is unused
-    if ((e = skv::launch_attn_tc(tq, tkd, tvd, tk, tv, tq, ta, d, st)) != cudaSuccess) return launch_err(h, e, "decode");
+    if ((e = skv::launch_attn_tc(tq, tkd, tvd, tk, tv, ta, d, st)) != cudaSuccess) return launch_err(h, e, "decode");
     sc.done();
   }
   if (split > 1) {
