@@ -54,8 +54,9 @@ struct AttnSmem {
   static constexpr int kQ = 0;                             // Q tiles A, B
   static constexpr int kKV = 2 * kTileBytes;               // ring
   static constexpr int kBar = kKV + kSlots * kTileBytes;
-  // q_full, kv_full[kSlots], kv_empty[kSlots], s_full[2], p_full[2], o_done[2], done, pv_done
-  static constexpr int kNumBars = 1 + 2 * kSlots + 6 + 1 + 1;
+  // q_full (tile A), kv_full[kSlots], kv_empty[kSlots], s_full[2], p_full[2], o_done[2], done, pv_done,
+  // q_full (tile B)
+  static constexpr int kNumBars = 1 + 2 * kSlots + 6 + 1 + 1 + 1;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4;
@@ -119,7 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nB = tB.valid ? max(0, min(ke, tB.nk) - kb) : 0;
   const int n_load = max(nA, nB);
 
-  const uint32_t bar_q = sb + L::kBar;
+  const uint32_t bar_q = sb + L::kBar;  // Q tile A
   auto bar_kvfull = [&](int sl) { return sb + L::kBar + 8u * (1 + sl); };
   auto bar_kvempty = [&](int sl) { return sb + L::kBar + 8u * (1 + kSlots + sl); };
   auto bar_sfull = [&](int x) { return sb + L::kBar + 8u * (1 + 2 * kSlots + x); };
@@ -127,6 +128,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar_odone = [&](int x) { return sb + L::kBar + 8u * (5 + 2 * kSlots + x); };
   const uint32_t bar_done = sb + L::kBar + 8u * (7 + 2 * kSlots);
   const uint32_t bar_pvdone = sb + L::kBar + 8u * (8 + 2 * kSlots);
+  const uint32_t bar_qb = sb + L::kBar + 8u * (9 + 2 * kSlots);  // Q tile B
   // With no keys for tile B in this CTA (a lone query tile: decode, or the
   // last tile of an odd count), tile A double-buffers S in the TMEM columns of
   // S_B: S(j+1) is computed while the softmax of tile j runs.
@@ -143,6 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tm_kf);
     tma_prefetch_desc(&tm_vf);
     mbar_init(bar_q, 1);
+    mbar_init(bar_qb, 1);
     for (int sl = 0; sl < kSlots; ++sl) {
       mbar_init(bar_kvfull(sl), 1);
       mbar_init(bar_kvempty(sl), 1);
@@ -175,15 +178,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const int nq = (nA > 0 ? 1 : 0) + (nB > 0 ? 1 : 0);
-      if (nq) {
-        mbar_arrive_expect_tx(bar_q, nq * L::kAtoms * a.q_rows * 128);
-        for (int at = 0; at < L::kAtoms; ++at) {
-          if (nA > 0) tma_load_4d(sb + L::kQ + at * L::kAtomBytes, &tm_q, bar_q, at * 64, tA.h, tA.i0, s);
-          if (nB > 0)
-            tma_load_4d(sb + L::kQ + L::kTileBytes + at * L::kAtomBytes, &tm_q, bar_q, at * 64, tB.h, tB.i0, s);
-        }
-      }
+      // Load order Q_A, K_0, Q_B, V_0, ...: S_A(0) needs only the first two
+      auto load_q = [&](int x) {
+        const uint32_t bar = x == 0 ? bar_q : bar_qb;
+        const TileInfo& ti = x == 0 ? tA : tB;
+        mbar_arrive_expect_tx(bar, L::kAtoms * a.q_rows * 128);
+        for (int at = 0; at < L::kAtoms; ++at)
+          tma_load_4d(sb + L::kQ + x * L::kTileBytes + at * L::kAtomBytes, &tm_q, bar, at * 64, ti.h, ti.i0, s);
+      };
+      if (nA > 0) load_q(0);
+      bool qb_issued = false;
       int issued = 0;
       for (int idx = 0; idx < 2 * n_load; ++idx) {
         const int sl = idx % kSlots;
@@ -199,8 +203,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           else tma_load_4d(dst + at * L::kAtomBytes, is_v ? &tm_vf : &tm_kf, bar_kvfull(sl), at * 64, g, r0, s);
         }
         issued = idx + 1;
+        if (idx == 0 && nB > 0) {
+          load_q(1);
+          qb_issued = true;
+        }
       }
-      if (nq) drain_wait(bar_q, 0, a.err);
+      if (nA > 0) drain_wait(bar_q, 0, a.err);
+      if (qb_issued) drain_wait(bar_qb, 0, a.err);
       for (int idx = (issued > kSlots ? issued - kSlots : 0); idx < issued; ++idx)
         drain_wait(bar_kvfull(idx % kSlots), (idx / kSlots) & 1, a.err);
     }
@@ -239,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ts(d_tmem, a_tmem + kk * 8, dv + (uint64_t)((kk * 2048) >> 4), id_o, (j > 0 || kk > 0) ? 1u : 0u);
         if (j == nX[x] - 1) mma_commit(bar_odone(x));
       };
-      bool ok = mbar_wait(bar_q, 0, a.err, kErrWaitLoad, abort_flag, wait_lim) && wait_slot(0);
+      bool ok = wait_slot(0) && (nA == 0 || mbar_wait(bar_q, 0, a.err, kErrWaitLoad, abort_flag, wait_lim));
       if (dbuf) {
         // S of tile j goes to buffer j & 1 (the S columns of tile A or B); the
         // softmax of tile j overlaps S(j+1).  The tensor pipe runs MMAs in
@@ -284,8 +293,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) {
         fence_after_sync();
         if (nA > 0) issue_s(0, 0);
-        if (nB > 0) issue_s(1, 0);
-        mma_commit(bar_kvempty(0));
+        if (nB > 0 && (ok = mbar_wait(bar_qb, 0, a.err, kErrWaitLoad, abort_flag, wait_lim))) {
+          fence_after_sync();
+          issue_s(1, 0);
+        }
+        if (ok) mma_commit(bar_kvempty(0));
       }
       // Ring order of tiles: K_0, V_0, K_1, V_1, ...; each slot is released
       // (kv_empty) after the last MMA reading it, in the same order.
@@ -467,10 +479,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int jj = 0; jj < 16; ++jj)
               pk[jj] = pack_bf16x2(__uint_as_float(v[2 * jj]) * inv, __uint_as_float(v[2 * jj + 1]) * inv);
             if (row_ok) {
-              uint4* dst = reinterpret_cast<uint4*>(a.o_part + prow * D + c0 * 32);
+              const long long plane = ((long long)(s * a.Hq + h) * a.n_split + sp);
 #pragma unroll
               for (int q4 = 0; q4 < 4; ++q4)
-                dst[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+                *reinterpret_cast<uint4*>(a.o_part + part_offset(plane, c0 * 4 + q4, i, a.T, D)) =
+                    make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
             }
           }
         }
@@ -490,7 +503,7 @@ template <int D>
 __global__ void __launch_bounds__(256) attn_combine_kernel(MergeArgs a) {
   pdl_wait();
   pdl_trigger();
-  merge_chunk<D>(a, blockIdx.x * blockDim.x + threadIdx.x);
+  merge_chunk<D>(a, (long long)blockIdx.x * blockDim.x + threadIdx.x);
 }
 
 // Merge of n_split float32 partials (O/l and log2-sum-exp per split): thread
@@ -598,7 +611,7 @@ MergeArgs merge_args(const AttnTcArgs& a, int d) {
 cudaError_t launch_attn_combine(const AttnTcArgs& a, int d, cudaStream_t st, bool pdl) {
   const MergeArgs m = merge_args(a, d);
   const long long rows = (long long)a.S * a.Hq * a.T;
-  const int blocks = (int)((rows * (d / 8) + 255) / 256);
+  const int blocks = (int)((merge_threads(rows, d) + 255) / 256);
   if (d == 128) return launch_kernel(attn_combine_kernel<128>, dim3(blocks), dim3(256), 0, st, pdl, m);
   return launch_kernel(attn_combine_kernel<64>, dim3(blocks), dim3(256), 0, st, pdl, m);
 }

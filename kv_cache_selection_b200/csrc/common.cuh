@@ -84,7 +84,7 @@ struct MergeArgs {
   int out_row;
   float* lse;                    // [S][Hq][T] natural log, may be null
   long long lse_s;
-  const __nv_bfloat16* o_part;   // [S][Hq][n_split][T][d] O/l per split
+  const __nv_bfloat16* o_part;   // O/l per split: planes [S][Hq][n_split] of [d/8][T][8]
   const float* ml_part;          // [S][Hq][n_split][T] log2-sum-exp
   int S, Hq, T, n_split, d;
 };

@@ -80,8 +80,8 @@ struct AttnTcArgs {
   int out_row;        // Hq * d
   float* lse;         // [S][Hq][T] natural log, may be null
   long long lse_s;
-  __nv_bfloat16* o_part;  // [S][Hq][n_split][T][d] O/l per split (n_split > 1)
-  float* o_part32;    // same layout in float32; used instead of o_part when set
+  __nv_bfloat16* o_part;  // O/l per split (n_split > 1): planes [S][Hq][n_split] of [d/8][T][8]
+  float* o_part32;    // [S][Hq][n_split][T][d] in float32; used instead of o_part when set
   float* ml_part;     // [S][Hq][n_split][T] log2-sum-exp
   int m, T, Hq, Hkv, causal, S;
   int n_it, n_pairs, n_split, nC, nF;

@@ -92,7 +92,7 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
   pdl_trigger();
   if ((int)blockIdx.x >= a.n_sel_blocks) {
     // extra blocks: merge of the attention's key-split partials
-    const int t = (blockIdx.x - a.n_sel_blocks) * kSelThreads + threadIdx.x;
+    const long long t = (long long)(blockIdx.x - a.n_sel_blocks) * kSelThreads + threadIdx.x;
     if (a.mrg.d == 128) merge_chunk<128>(a.mrg, t);
     else merge_chunk<64>(a.mrg, t);
     return;
@@ -441,7 +441,7 @@ cudaError_t launch_select(const SelectArgs& a_in, int S, cudaStream_t st, bool p
   const int n_groups = a.global ? 1 : a.Hkv;
   a.n_sel_blocks = n_groups * S;
   if (a.mrg.n_split > 1) {
-    const long long mrg_threads = (long long)a.mrg.S * a.mrg.Hq * a.mrg.T * (a.mrg.d / 8);
+    const long long mrg_threads = merge_threads((long long)a.mrg.S * a.mrg.Hq * a.mrg.T, a.mrg.d);
     a.n_mrg_blocks = (int)((mrg_threads + kSelThreads - 1) / kSelThreads);
   } else {
     a.n_mrg_blocks = 0;
