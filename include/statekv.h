@@ -295,14 +295,6 @@ int statekv_step_noalloc(int Hq, int Hkv, int d, int T, int B, int dtype, int ma
                          int32_t* posc_new, float* scorec_new, void* kd, void* vd,
                          int32_t* posd, int d_len, int max_tok, void* stream);
 
-/* Self-test of the FMA-pipe exponential the kernels may use in place of the
- * MUFU unit for part of their exponentials: y[i] = 2^x[i] for n float32
- * values (device pointers) on `stream`.  The paper has no counterpart; tests
- * compare it with CUDA's exp2f (maximum relative error 7.5e-5 for
- * -125 <= x <= 127; below -125 a non-negative value under 2^-124).  Errors (message in statekv_last_error(NULL)):
- * INVALID_ARG, CUDA. */
-int statekv_selftest_exp2(const float* x, float* y, int n, void* stream);
-
 #ifdef __cplusplus
 }
 #endif

@@ -29,9 +29,6 @@ namespace {
 using namespace tc;
 
 constexpr int kStages = 4;
-// Every kFmaExpEvery-th exponential runs on the FMA pipe (exp2_fma) instead of
-// MUFU, which otherwise issues all of them (0: none).
-constexpr int kFmaExpEvery = 0;
 constexpr int kGroups = 3;                      // epilogue warpgroups (take chunks round robin)
 constexpr int kEpiWarps = 4 * kGroups;
 constexpr int kThreads = 128 + 32 * kEpiWarps;  // warpgroup 0: producer, MMA, two idle warps
@@ -69,14 +66,10 @@ __device__ __forceinline__ void score_cols16(const uint32_t (&rr)[16], const flo
 #pragma unroll
   for (int j4 = 0; j4 < 4; ++j4) {
     const float4 lv = l4[j4];  // -lse2 of 4 columns
-    auto ex = [](int e, float x) {
-      return (kFmaExpEvery > 0 && e % (kFmaExpEvery > 0 ? kFmaExpEvery : 1) == kFmaExpEvery - 1) ? exp2_fma(x)
-                                                                                              : ex2_approx(x);
-    };
-    float p0 = ex(4 * j4 + 0, fmaf(__uint_as_float(rr[4 * j4 + 0]), scale_log2, lv.x));
-    float p1 = ex(4 * j4 + 1, fmaf(__uint_as_float(rr[4 * j4 + 1]), scale_log2, lv.y));
-    float p2 = ex(4 * j4 + 2, fmaf(__uint_as_float(rr[4 * j4 + 2]), scale_log2, lv.z));
-    float p3 = ex(4 * j4 + 3, fmaf(__uint_as_float(rr[4 * j4 + 3]), scale_log2, lv.w));
+    float p0 = ex2_approx(fmaf(__uint_as_float(rr[4 * j4 + 0]), scale_log2, lv.x));
+    float p1 = ex2_approx(fmaf(__uint_as_float(rr[4 * j4 + 1]), scale_log2, lv.y));
+    float p2 = ex2_approx(fmaf(__uint_as_float(rr[4 * j4 + 2]), scale_log2, lv.z));
+    float p3 = ex2_approx(fmaf(__uint_as_float(rr[4 * j4 + 3]), scale_log2, lv.w));
     if (need_mask) {
       // frame token `key` is seen by rows i >= key (frame-causal); rows past T do not exist
       const int i = i0 + 4 * j4;

@@ -311,29 +311,6 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int* er
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
-// 2^x on the FMA pipe, for kernels whose exponentials outnumber what the MUFU
-// unit issues (16 per clock per SM).  Cody-Waite style range reduction: adding
-// 1.5 * 2^23 rounds x to the nearest integer j in the low mantissa bits of t,
-// f = x - j lies in [-1/2, 1/2]; 2^f comes from a degree-3 polynomial whose
-// coefficients were fitted here by Lawson's iteratively reweighted least
-// squares for minimal maximum relative error on [-1/2, 1/2] (7.5e-5; the fit
-// is reproduced by kv_cache_selection_b200/fit_exp2.py); 2^j is applied by
-// adding j to the exponent field.  Relative error 7.5e-5 for -125 <= x <=
-// 127.  Inputs below -126 (and -inf) are raised to -126, so that j >= -126
-// keeps the exponent field non-negative: below -125 the result is a
-// non-negative value under 2^-124 (not 0; callers that need exact zeros mask
-// them).
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -126.f);
-  const float t = x + 12582912.f;  // 1.5 * 2^23
-  const float j = t - 12582912.f;
-  const float f = x - j;
-  float p = fmaf(f, 0.05517132207751274f, 0.24261054396629333f);
-  p = fmaf(f, p, 0.6932609677314758f);
-  p = fmaf(f, p, 0.9999281167984009f);
-  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
-}
-
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

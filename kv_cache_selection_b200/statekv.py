@@ -55,7 +55,6 @@ _SIGS = {
     "statekv_last_error": (ctypes.c_char_p, [_vp]),
     "statekv_step_noalloc": (_i, [_i] * 8 + [_vp] * 7 + [_i] + [_vp] * 8 + [_i, _i, _vp]),
     "statekv_decode": (_i, [_vp, _i, _vp, _vp, _vp, _i, _vp, _vp, _vp]),
-    "statekv_selftest_exp2": (_i, [_vp, _vp, _i, _vp]),
     "full_causal_prefill": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp]),
     "full_causal_prefill_batched": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp]),
 }
