@@ -108,6 +108,7 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
   //    (ascending group), written out as the pool scores and staged as bits
   const float* __restrict__ part = a.part + s * a.part_s;
   float* pool_score = a.pool_score + s * a.part_s + (long long)G0 * a.part_g;
+  uint32_t tmin = 0xffffffffu, tmax = 0u;  // span of this thread's staged values (first level)
   if ((a.part_g & 3) == 0 && (reinterpret_cast<uintptr_t>(part) & 15) == 0) {
     // four consecutive candidates per thread and group as one 16-byte load
     const int n4 = (L + 3) / 4;
@@ -139,12 +140,27 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
           v.w += x[u].w;
         }
       }
-      const float vv[4] = {v.x, v.y, v.z, v.w};
+      if (full && (reinterpret_cast<uintptr_t>(pool_score) & 15) == 0) {
+        *reinterpret_cast<float4*>(pool_score + j0) = v;
+        if (!a.recency) {
+          const uint4 b4 = make_uint4(score_bits(v.x), score_bits(v.y), score_bits(v.z), score_bits(v.w));
+          *reinterpret_cast<uint4*>(su + j0) = b4;
+          tmin = min(min(tmin, min(b4.x, b4.y)), min(b4.z, b4.w));
+          tmax = max(max(tmax, max(b4.x, b4.y)), max(b4.z, b4.w));
+        }
+      } else {
+        const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        if (j0 + e < L) {
-          pool_score[j0 + e] = vv[e];
-          su[j0 + e] = score_bits(vv[e]);
+        for (int e = 0; e < 4; ++e) {
+          if (j0 + e < L) {
+            pool_score[j0 + e] = vv[e];
+            if (!a.recency) {
+              const uint32_t b = score_bits(vv[e]);
+              su[j0 + e] = b;
+              tmin = min(tmin, b);
+              tmax = max(tmax, b);
+            }
+          }
         }
       }
     }
@@ -153,16 +169,35 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
       float v = 0.f;
       for (int g = G0; g < G1; ++g) v += __ldg(part + (long long)g * a.part_g + j);
       pool_score[j] = v;
-      su[j] = score_bits(v);
+      if (!a.recency) {
+        const uint32_t b = score_bits(v);
+        su[j] = b;
+        tmin = min(tmin, b);
+        tmax = max(tmax, b);
+      }
     }
   }
   if (a.recency) {
     // recency retention ranks by position: the bit pattern of a non-negative
-    // int32 orders like its value, and positions are distinct (no ties)
+    // int32 orders like its value, and positions are distinct (no ties).  The
+    // score loops above leave su alone in this mode: each word of su is written
+    // by one thread only (they map candidates to threads differently).
     const int* __restrict__ pos_c = a.pos_c + ((long long)s * a.Hkv + G0) * a.B;
     const int* __restrict__ pos_f = a.pos_f + (long long)s * a.T;
-    for (int j = threadIdx.x; j < L; j += kSelThreads)
-      su[j] = (uint32_t)max(j < a.m ? __ldg(pos_c + j) : __ldg(pos_f + (j - a.m)), 0);
+    for (int j = threadIdx.x; j < L; j += kSelThreads) {
+      const uint32_t b = (uint32_t)max(j < a.m ? __ldg(pos_c + j) : __ldg(pos_f + (j - a.m)), 0);
+      su[j] = b;
+      tmin = min(tmin, b);
+      tmax = max(tmax, b);
+    }
+  }
+  // the first level of the threshold search takes its span from here
+  reinterpret_cast<uint4*>(sh.hist)[threadIdx.x] = make_uint4(0u, 0u, 0u, 0u);
+  tmin = warp_min_u32(tmin);
+  tmax = warp_max_u32(tmax);
+  if (lane == 0) {
+    sh.warp_a[warp] = tmin;
+    sh.warp_b[warp] = tmax;
   }
   __syncthreads();
   if (a.B <= 0) return;  // nothing is kept (block-uniform)
@@ -174,24 +209,27 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
   if (!keep_all) {
     uint32_t lo = 0, hi = 0xffffffffu;  // span of the values still in play (inclusive)
     uint32_t need = (uint32_t)a.B;      // how many of them are kept
-    for (;;) {
+    for (int level = 0;; ++level) {
       // exact span of the values in play; the histogram is cleared meanwhile
+      // (the first level's span and cleared histogram come from the load)
       uint32_t vmin = 0xffffffffu, vmax = 0u;
-      for (int j = threadIdx.x; j < L; j += kSelThreads) {
-        const uint32_t u = su[j];
-        if (u >= lo && u <= hi) {
-          vmin = min(vmin, u);
-          vmax = max(vmax, u);
+      if (level > 0) {
+        for (int j = threadIdx.x; j < L; j += kSelThreads) {
+          const uint32_t u = su[j];
+          if (u >= lo && u <= hi) {
+            vmin = min(vmin, u);
+            vmax = max(vmax, u);
+          }
         }
+        reinterpret_cast<uint4*>(sh.hist)[threadIdx.x] = make_uint4(0u, 0u, 0u, 0u);
+        vmin = warp_min_u32(vmin);
+        vmax = warp_max_u32(vmax);
+        if (lane == 0) {
+          sh.warp_a[warp] = vmin;
+          sh.warp_b[warp] = vmax;
+        }
+        __syncthreads();
       }
-      reinterpret_cast<uint4*>(sh.hist)[threadIdx.x] = make_uint4(0u, 0u, 0u, 0u);
-      vmin = warp_min_u32(vmin);
-      vmax = warp_max_u32(vmax);
-      if (lane == 0) {
-        sh.warp_a[warp] = vmin;
-        sh.warp_b[warp] = vmax;
-      }
-      __syncthreads();
       if (warp == 0) {
         const uint32_t m0 = warp_min_u32(sh.warp_a[lane]), m1 = warp_max_u32(sh.warp_b[lane]);
         if (lane == 0) {
@@ -329,6 +367,10 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
   uint32_t eq_seen = packed >> 16;                                      // tied candidates before j_lo
   int dst = (int)(packed & 0xffffu) + (int)min(eq_seen, need_eq);       // kept candidates before j_lo
   int32_t* idx = a.idx + ((long long)s * a.Hkv + G0) * a.B;
+  // Scattered 4-byte global stores cost several thousand cycles here; when B
+  // fits the (now unused) histogram, the kept indices are placed there and
+  // copied out with coalesced stores.
+  const bool stage = a.B <= kBins;
   for (int j = j_lo; j < j_hi; ++j) {
     bool keep;
     if (keep_all) {
@@ -339,9 +381,17 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
       if (u == tau) keep = eq_seen++ < need_eq;
     }
     if (keep) {
-      if (dst < a.B) idx[dst] = j;
+      if (dst < a.B) {
+        if (stage) sh.hist[dst] = (uint32_t)j;
+        else idx[dst] = j;
+      }
       ++dst;
     }
+  }
+  if (stage) {
+    __syncthreads();
+    const int n_kept = min(a.B, L);
+    for (int r = threadIdx.x; r < n_kept; r += kSelThreads) idx[r] = (int32_t)sh.hist[r];
   }
 }
 
