@@ -121,13 +121,17 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k,
 /* statekv_prefill_frame with HOST buffers: q, k, v, pos are read from and out
  * is written to host memory (same layouts; page-locked memory makes the copies
  * asynchronous, pageable memory is accepted).  The call copies the inputs into
- * one of two library-owned staging sets on a library-owned copy stream (so the
- * copies of call n+1 overlap the step of call n), makes `stream` wait for them,
- * enqueues the step and the device-to-host copy of out on `stream`.  When
- * `stream` has reached the end of the call, the inputs have been read and out
- * is complete (synchronise the stream before reading out or reusing the input
- * buffers).  The first call creates the staging buffers, the copy stream and
- * its events (synchronous).  Errors: as statekv_prefill_frame. */
+ * one of two library-owned staging sets on a library-owned copy stream, runs
+ * the step on a library-owned compute stream once they have arrived, and
+ * makes `stream` wait for the step and copy out back.  So the copies of call
+ * n+1 and the copy-out of call n overlap the steps.  When `stream` has reached
+ * the end of the call, the inputs have been read and out is complete
+ * (synchronise the stream before reading out or reusing the input buffers).
+ * A layer's frames may come through both entry points: the library orders a
+ * layer's step after its previous one (a host-buffer step after device-buffer
+ * steps enqueued on `stream` before it).  The first call creates the staging
+ * buffers, the two streams and their events (synchronous).  Errors: as
+ * statekv_prefill_frame. */
 int statekv_prefill_frame_host(statekv_t h, int layer, const void* q, const void* k,
                                const void* v, const int32_t* pos, void* out, void* stream);
 

@@ -29,6 +29,12 @@ thread_local std::string g_free_error;  // errors of calls without a handle
 struct LayerState {
   bool ready = false;
   int frames = 0;
+  // entry point of the layer's last step (0 none, 1 device buffers on the
+  // caller's stream, 2 host buffers on the library's compute stream) and the
+  // completion of its last host-buffer step, which orders the layer's next
+  // device-buffer step after it
+  int last_entry = 0;
+  cudaEvent_t ev_host_done = nullptr;
   int m = 0;    // current C length
   int cur = 0;  // index of the current C buffer
   void* kc[2] = {nullptr, nullptr};
@@ -72,8 +78,11 @@ struct statekv_handle {
   int32_t* stage_pos[2] = {nullptr, nullptr};
   int stage_next = 0;
   cudaStream_t copy_stream = nullptr;
+  cudaStream_t compute_stream = nullptr;  // the steps of host-buffer calls
   cudaEvent_t ev_h2d[2] = {nullptr, nullptr};   // inputs of set b are on the device
+  cudaEvent_t ev_step_done[2] = {nullptr, nullptr};  // the step that reads set b is done
   cudaEvent_t ev_stage_free[2] = {nullptr, nullptr};  // the step and copy-out of set b are done
+  cudaEvent_t ev_caller = nullptr;  // tail of the caller's stream (device-buffer steps before a host call)
   // key-split partials of statekv_decode (float32), grown on demand
   float* dec_o = nullptr;
   float* dec_ml = nullptr;
@@ -401,8 +410,10 @@ int statekv_reserve_layers(statekv_t h, int n_layers) {
   return STATEKV_OK;
 }
 
-int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, const void* v,
-                          const int32_t* pos, void* out, void* stream) {
+namespace {
+// One frame of one layer on `stream` (both entry points).
+int prefill_step(statekv_t h, int layer, const void* q, const void* k, const void* v, const int32_t* pos,
+                 void* out, void* stream) {
   if (!h) return set_err(nullptr, STATEKV_ERR_INVALID_ARG, "null handle");
   if (!q || !k || !v || !pos || !out)
     return set_err(h, STATEKV_ERR_INVALID_ARG, "null input/output pointer");
@@ -614,6 +625,21 @@ int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, 
   h->last_layer = layer;
   return STATEKV_OK;
 }
+}  // namespace
+
+int statekv_prefill_frame(statekv_t h, int layer, const void* q, const void* k, const void* v,
+                          const int32_t* pos, void* out, void* stream) {
+  if (!h) return set_err(nullptr, STATEKV_ERR_INVALID_ARG, "null handle");
+  LayerState* L = (layer >= 0 && (size_t)layer < h->layers.size()) ? &h->layers[layer] : nullptr;
+  if (L && L->last_entry == 2 && L->ev_host_done) {
+    // the layer's previous step came through the host-buffer call
+    const cudaError_t e = cudaStreamWaitEvent(static_cast<cudaStream_t>(stream), L->ev_host_done, 0);
+    if (e != cudaSuccess) return set_err(h, STATEKV_ERR_CUDA, "stream wait failed: %s", cudaGetErrorString(e));
+  }
+  const int rc = prefill_step(h, layer, q, k, v, pos, out, stream);
+  if (rc == STATEKV_OK) h->layers[layer].last_entry = 1;
+  return rc;
+}
 
 int statekv_prefill_frame_host(statekv_t h, int layer, const void* q, const void* k, const void* v,
                                const int32_t* pos, void* out, void* stream) {
@@ -631,35 +657,55 @@ int statekv_prefill_frame_host(statekv_t h, int layer, const void* q, const void
           (rc = dev_alloc(h, &h->stage_v[b], kb)) || (rc = dev_alloc(h, &h->stage_out[b], qb)) ||
           (rc = dev_alloc(h, (void**)&h->stage_pos[b], pb)))
         return rc;
-    if ((e = cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking)) != cudaSuccess)
-      return set_err(h, STATEKV_ERR_CUDA, "copy stream: %s", cudaGetErrorString(e));
+    if ((e = cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaStreamCreateWithFlags(&h->compute_stream, cudaStreamNonBlocking)) != cudaSuccess)
+      return set_err(h, STATEKV_ERR_CUDA, "staging streams: %s", cudaGetErrorString(e));
     for (int b = 0; b < 2; ++b)
       if ((e = cudaEventCreateWithFlags(&h->ev_h2d[b], cudaEventDisableTiming)) != cudaSuccess ||
+          (e = cudaEventCreateWithFlags(&h->ev_step_done[b], cudaEventDisableTiming)) != cudaSuccess ||
           (e = cudaEventCreateWithFlags(&h->ev_stage_free[b], cudaEventDisableTiming)) != cudaSuccess)
         return set_err(h, STATEKV_ERR_CUDA, "staging events: %s", cudaGetErrorString(e));
+    if ((e = cudaEventCreateWithFlags(&h->ev_caller, cudaEventDisableTiming)) != cudaSuccess)
+      return set_err(h, STATEKV_ERR_CUDA, "staging events: %s", cudaGetErrorString(e));
   }
   // the step's own refusals, checked before anything is enqueued
   if (layer < 0) return set_err(h, STATEKV_ERR_INVALID_ARG, "negative layer %d", layer);
   if ((size_t)layer < h->layers.size() && h->layers[layer].ready && h->layers[layer].frames >= h->max_frames)
     return set_err(h, STATEKV_ERR_CAPACITY, "layer %d already holds max_frames=%d frames", layer, h->max_frames);
+  LayerState* L;
+  if ((rc = get_layer(h, layer, &L))) return rc;
+  if (!L->ev_host_done && (e = cudaEventCreateWithFlags(&L->ev_host_done, cudaEventDisableTiming)) != cudaSuccess)
+    return set_err(h, STATEKV_ERR_CUDA, "layer event: %s", cudaGetErrorString(e));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaStream_t cs = h->compute_stream;
   const int b = h->stage_next;
-  // The inputs of this call go to staging set b on the copy stream once the
-  // step that last read set b is done, so they can arrive while the previous
-  // call's step still runs; the step waits for them, then copies out back on
-  // the caller's stream.
+  // Three streams: the inputs of this call go to staging set b on the copy
+  // stream once set b's last step and copy-out are done; the step runs on the
+  // library's compute stream once they have arrived; `stream` waits for the
+  // step and copies out back.  So the copies of call n+1 and the copy-out of
+  // call n overlap the steps of calls n and n+1, and when `stream` has reached
+  // the end of this call out is complete.
   if ((e = cudaStreamWaitEvent(h->copy_stream, h->ev_stage_free[b], 0)) != cudaSuccess ||
       (e = cudaMemcpyAsync(h->stage_q[b], q, qb, cudaMemcpyHostToDevice, h->copy_stream)) != cudaSuccess ||
       (e = cudaMemcpyAsync(h->stage_k[b], k, kb, cudaMemcpyHostToDevice, h->copy_stream)) != cudaSuccess ||
       (e = cudaMemcpyAsync(h->stage_v[b], v, kb, cudaMemcpyHostToDevice, h->copy_stream)) != cudaSuccess ||
       (e = cudaMemcpyAsync(h->stage_pos[b], pos, pb, cudaMemcpyHostToDevice, h->copy_stream)) != cudaSuccess ||
       (e = cudaEventRecord(h->ev_h2d[b], h->copy_stream)) != cudaSuccess ||
-      (e = cudaStreamWaitEvent(st, h->ev_h2d[b], 0)) != cudaSuccess)
+      (e = cudaStreamWaitEvent(cs, h->ev_h2d[b], 0)) != cudaSuccess)
     return set_err(h, STATEKV_ERR_CUDA, "host-to-device copy failed: %s", cudaGetErrorString(e));
-  rc = statekv_prefill_frame(h, layer, h->stage_q[b], h->stage_k[b], h->stage_v[b], h->stage_pos[b],
-                             h->stage_out[b], stream);
+  if (L->last_entry == 1) {
+    // the layer's previous step came through the device-buffer call on the
+    // caller's stream
+    if ((e = cudaEventRecord(h->ev_caller, st)) != cudaSuccess || (e = cudaStreamWaitEvent(cs, h->ev_caller, 0)) != cudaSuccess)
+      return set_err(h, STATEKV_ERR_CUDA, "stream wait failed: %s", cudaGetErrorString(e));
+  }
+  rc = prefill_step(h, layer, h->stage_q[b], h->stage_k[b], h->stage_v[b], h->stage_pos[b], h->stage_out[b], cs);
   if (rc) return rc;
-  if ((e = cudaMemcpyAsync(out, h->stage_out[b], qb, cudaMemcpyDeviceToHost, st)) != cudaSuccess ||
+  L->last_entry = 2;
+  if ((e = cudaEventRecord(h->ev_step_done[b], cs)) != cudaSuccess ||
+      (e = cudaEventRecord(L->ev_host_done, cs)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(st, h->ev_step_done[b], 0)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(out, h->stage_out[b], qb, cudaMemcpyDeviceToHost, st)) != cudaSuccess ||
       (e = cudaEventRecord(h->ev_stage_free[b], st)) != cudaSuccess)
     return set_err(h, STATEKV_ERR_CUDA, "device-to-host copy failed: %s", cudaGetErrorString(e));
   h->stage_next = b ^ 1;
@@ -900,9 +946,14 @@ int statekv_destroy(statekv_t h) {
   }
   for (int b = 0; b < 2; ++b) {
     if (h->ev_h2d[b]) cudaEventDestroy(h->ev_h2d[b]);
+    if (h->ev_step_done[b]) cudaEventDestroy(h->ev_step_done[b]);
     if (h->ev_stage_free[b]) cudaEventDestroy(h->ev_stage_free[b]);
   }
+  if (h->ev_caller) cudaEventDestroy(h->ev_caller);
+  for (auto& L : h->layers)
+    if (L.ev_host_done) cudaEventDestroy(L.ev_host_done);
   if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
+  if (h->compute_stream) cudaStreamDestroy(h->compute_stream);
   for (cudaEvent_t e : h->ev_free) cudaEventDestroy(e);
   for (void* p : h->allocs) cudaFree(p);
   if (h->dec_o) cudaFree(h->dec_o);

@@ -346,6 +346,47 @@ def test_host_buffer_entry_parity(dtype):
 
 
 @cuda
+def test_host_and_device_entries_interleaved_without_synchronisation():
+    """One layer's frames through both entry points in turn, with no host
+    synchronisation between calls: the host-buffer steps run on the
+    library's compute stream, so the library must order each step after the
+    layer's previous one.  C, D and every frame's out equal those of a run
+    through the device-buffer call alone (bit for bit: same kernels)."""
+    S = _skv()
+    wl = Syn.workload("1b_layer", Hq=14, Hkv=2, d=64, T=256, B=512, frames=8)
+    dev = torch.device("cuda")
+    frames = [Syn.gen_frame(wl, n) for n in range(wl.frames)]
+    ref = S.StateKV(wl.Hq, wl.Hkv, wl.d, wl.T, wl.B, max_frames=wl.frames, dtype="bf16")
+    ref_out = [ref.prefill_frame(0, *(t.to(dev) for t in fr)).clone() for fr in frames]
+    torch.cuda.synchronize()
+    h = S.StateKV(wl.Hq, wl.Hkv, wl.d, wl.T, wl.B, max_frames=wl.frames, dtype="bf16")
+    outs, keep = [], []  # host buffers stay alive until the final synchronisation
+    for n, fr in enumerate(frames):
+        if n % 3 == 1 or n % 3 == 2:  # pattern: device, host, host, device, host, host, ...
+            q, k, v, pos = (t.cpu().pin_memory() for t in fr)
+            out = torch.empty_like(q).pin_memory()
+            h.prefill_frame_host(0, q, k, v, pos, out)
+            keep.append((q, k, v, pos))
+            outs.append(out)
+        else:
+            dev_in = [t.to(dev) for t in fr]
+            keep.append(dev_in)
+            outs.append(h.prefill_frame(0, *dev_in))
+    torch.cuda.synchronize()
+    for n in range(wl.frames):
+        assert torch.equal(outs[n].to(dev), ref_out[n]), f"out of frame {n}"
+    Ca, Cb = h.get_compressed(0), ref.get_compressed(0)
+    assert Ca["len"] == Cb["len"]
+    for key in ("k", "v", "pos", "score"):
+        assert torch.equal(Ca[key], Cb[key]), key
+    Da, Db = h.get_detailed(0), ref.get_detailed(0)
+    for key in ("k", "v", "pos"):
+        assert torch.equal(Da[key], Db[key]), key
+    h.close()
+    ref.close()
+
+
+@cuda
 @pytest.mark.parametrize("dtype,Hq,Hkv,select", [("f32", 12, 12, "global"), ("bf16", 20, 10, "global"),
                                                 ("bf16", 20, 10, "per_kv_head")])
 def test_more_than_eight_kv_heads(dtype, Hq, Hkv, select):
