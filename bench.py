@@ -281,10 +281,30 @@ def run_ours(args, wl):
         esize = 2 if wl.dtype == "bf16" else 4
         h2d = (wl.T * wl.Hq * wl.d + 2 * wl.T * wl.Hkv * wl.d) * esize + wl.T * 4
         d2h = wl.T * wl.Hq * wl.d * esize
+        # the PCIe copies alone (same bytes, pinned memory, one direction at a
+        # time): the floor that the end-to-end step time is set against
+        hx = torch.empty(h2d, dtype=torch.uint8).pin_memory()
+        dx = torch.empty(max(h2d, d2h), dtype=torch.uint8, device=dev)
+        cs = torch.cuda.Stream()
+        link = {}
+        for name, n_b, fn in (("h2d", h2d, lambda: dx[:h2d].copy_(hx, non_blocking=True)),
+                              ("d2h", d2h, lambda: hx[:d2h].copy_(dx[:d2h], non_blocking=True))):
+            with torch.cuda.stream(cs):
+                for _ in range(3):
+                    fn()
+                c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                c0.record()
+                for _ in range(20):
+                    fn()
+                c1.record()
+            c1.synchronize()
+            link[name + "_us"] = round(c0.elapsed_time(c1) / 20 * 1e3, 2)
+            link[name + "_gbs"] = round(n_b / (c0.elapsed_time(c1) / 20 * 1e-3) / 1e9, 2)
         e2e = {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / K, 5),
                "path": "statekv_prefill_frame_host (pinned host buffers; the library stages the copies)",
-               "l2": "not flushed (host copies dominate)"}
+               "l2": "not flushed (host copies dominate)",
+               "pcie_copies_alone": link}
         he.close()
 
     # ---- host enqueue cost of one step (back-to-back calls, no synchronisation)
