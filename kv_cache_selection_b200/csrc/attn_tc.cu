@@ -407,22 +407,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // P = exp2(S*c - m_used) (masked entries hold -inf -> 0), as bf16 into
       // the first 64 columns of the same TMEM region
-      float ls0 = 0.f, ls1 = 0.f;
+      // (the scale-and-shift and the row sums in paired float32 instructions)
+      const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_used, -m_used);
+      float2 ls = make_float2(0.f, 0.f);
 #pragma unroll
       for (int c0 = 0; c0 < 4; ++c0) {
         uint32_t pk[16];
 #pragma unroll
         for (int jj = 0; jj < 16; ++jj) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(sv[c0 * 32 + 2 * jj]), c, -m_used));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(sv[c0 * 32 + 2 * jj + 1]), c, -m_used));
-          ls0 += p0;
-          ls1 += p1;
-          pk[jj] = pack_bf16x2(p0, p1);
+          const float2 x = ffma2(make_float2(__uint_as_float(sv[c0 * 32 + 2 * jj]),
+                                             __uint_as_float(sv[c0 * 32 + 2 * jj + 1])), c2, nm2);
+          const float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          ls = fadd2(ls, pp);
+          pk[jj] = pack_bf16x2(pp.x, pp.y);
         }
         tmem_st16(t_s + c0 * 16, pk);
       }
       tmem_st_wait();
-      l += ls0 + ls1;
+      l += ls.x + ls.y;
       fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_pfull(sbuf));

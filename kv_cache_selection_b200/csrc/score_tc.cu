@@ -66,10 +66,15 @@ __device__ __forceinline__ void score_cols16(const uint32_t (&rr)[16], const flo
 #pragma unroll
   for (int j4 = 0; j4 < 4; ++j4) {
     const float4 lv = l4[j4];  // -lse2 of 4 columns
-    float p0 = ex2_approx(fmaf(__uint_as_float(rr[4 * j4 + 0]), scale_log2, lv.x));
-    float p1 = ex2_approx(fmaf(__uint_as_float(rr[4 * j4 + 1]), scale_log2, lv.y));
-    float p2 = ex2_approx(fmaf(__uint_as_float(rr[4 * j4 + 2]), scale_log2, lv.z));
-    float p3 = ex2_approx(fmaf(__uint_as_float(rr[4 * j4 + 3]), scale_log2, lv.w));
+    const float2 sc2 = make_float2(scale_log2, scale_log2);
+    const float2 x01 = ffma2(make_float2(__uint_as_float(rr[4 * j4 + 0]), __uint_as_float(rr[4 * j4 + 1])), sc2,
+                             make_float2(lv.x, lv.y));
+    const float2 x23 = ffma2(make_float2(__uint_as_float(rr[4 * j4 + 2]), __uint_as_float(rr[4 * j4 + 3])), sc2,
+                             make_float2(lv.z, lv.w));
+    float p0 = ex2_approx(x01.x);
+    float p1 = ex2_approx(x01.y);
+    float p2 = ex2_approx(x23.x);
+    float p3 = ex2_approx(x23.y);
     if (need_mask) {
       // frame token `key` is seen by rows i >= key (frame-causal); rows past T do not exist
       const int i = i0 + 4 * j4;
@@ -78,10 +83,12 @@ __device__ __forceinline__ void score_cols16(const uint32_t (&rr)[16], const flo
       p2 = (i + 2 < T && (!diag || key <= i + 2)) ? p2 : 0.f;
       p3 = (i + 3 < T && (!diag || key <= i + 3)) ? p3 : 0.f;
     }
-    acc0 += p0;
-    acc1 += p1;
-    acc2 += p2;
-    acc3 += p3;
+    const float2 a01 = fadd2(make_float2(acc0, acc1), make_float2(p0, p1));
+    const float2 a23 = fadd2(make_float2(acc2, acc3), make_float2(p2, p3));
+    acc0 = a01.x;
+    acc1 = a01.y;
+    acc2 = a23.x;
+    acc3 = a23.y;
   }
 }
 
