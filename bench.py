@@ -273,8 +273,10 @@ def run_ours(args, wl):
             torch.distributed.barrier()
         torch.cuda.synchronize()
         e0.record()
+        th0 = time.perf_counter()
         for j in range(K):
             host_step(fill + W + j)
+        host_call_us = (time.perf_counter() - th0) / K * 1e6
         e1.record()
         torch.cuda.synchronize()
         e2e_value, e2e_ms = replica_throughput(K, e0.elapsed_time(e1), dev)
@@ -314,10 +316,31 @@ def run_ours(args, wl):
             n_b = h2d if name == "h2d" else d2h
             link[name + "_us"] = round(us, 2)
             link[name + "_gbs"] = round(n_b / (us * 1e-6) / 1e9, 2)
+        # both directions at once, on two streams
+        cs2 = torch.cuda.Stream()
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        c0.record()
+        cs.wait_event(c0)
+        cs2.wait_event(c0)
+        for _ in range(20):
+            with torch.cuda.stream(cs):
+                h2d_copy()
+            with torch.cuda.stream(cs2):
+                d2h_copy()
+        e_a, e_b = torch.cuda.Event(), torch.cuda.Event()
+        e_a.record(cs)
+        e_b.record(cs2)
+        torch.cuda.current_stream().wait_event(e_a)
+        torch.cuda.current_stream().wait_event(e_b)
+        c1.record()
+        c1.synchronize()
+        link["both_directions_us"] = round(c0.elapsed_time(c1) / 20 * 1e3, 2)
         e2e = {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / K, 5),
                "path": "statekv_prefill_frame_host (pinned host buffers; the library stages the copies)",
                "l2": "not flushed (host copies dominate)",
+               "host_us_per_call": round(host_call_us, 2),
                "pcie_copies_alone": link}
         he.close()
 

@@ -80,8 +80,8 @@ struct statekv_handle {
   cudaStream_t copy_stream = nullptr;
   cudaStream_t compute_stream = nullptr;  // the steps of host-buffer calls
   cudaEvent_t ev_h2d[2] = {nullptr, nullptr};   // inputs of set b are on the device
-  cudaEvent_t ev_step_done[2] = {nullptr, nullptr};  // the step that reads set b is done
-  cudaEvent_t ev_stage_free[2] = {nullptr, nullptr};  // the step and copy-out of set b are done
+  cudaEvent_t ev_step_done[2] = {nullptr, nullptr};  // the step that reads set b's inputs is done
+  cudaEvent_t ev_stage_free[2] = {nullptr, nullptr};  // the copy-out of set b's output is done
   cudaEvent_t ev_caller = nullptr;  // tail of the caller's stream (device-buffer steps before a host call)
   // key-split partials of statekv_decode (float32), grown on demand
   float* dec_o = nullptr;
@@ -680,18 +680,20 @@ int statekv_prefill_frame_host(statekv_t h, int layer, const void* q, const void
   cudaStream_t cs = h->compute_stream;
   const int b = h->stage_next;
   // Three streams: the inputs of this call go to staging set b on the copy
-  // stream once set b's last step and copy-out are done; the step runs on the
-  // library's compute stream once they have arrived; `stream` waits for the
-  // step and copies out back.  So the copies of call n+1 and the copy-out of
-  // call n overlap the steps of calls n and n+1, and when `stream` has reached
-  // the end of this call out is complete.
-  if ((e = cudaStreamWaitEvent(h->copy_stream, h->ev_stage_free[b], 0)) != cudaSuccess ||
+  // stream once set b's last step has read its inputs; the step runs on the
+  // library's compute stream once they have arrived and set b's last output
+  // has been copied out; `stream` waits for the step and copies out back.  So
+  // the copy-in of call n+1 and the copy-out of call n overlap the steps, the
+  // two directions overlap each other, and when `stream` has reached the end
+  // of this call out is complete.
+  if ((e = cudaStreamWaitEvent(h->copy_stream, h->ev_step_done[b], 0)) != cudaSuccess ||
       (e = cudaMemcpyAsync(h->stage_q[b], q, qb, cudaMemcpyHostToDevice, h->copy_stream)) != cudaSuccess ||
       (e = cudaMemcpyAsync(h->stage_k[b], k, kb, cudaMemcpyHostToDevice, h->copy_stream)) != cudaSuccess ||
       (e = cudaMemcpyAsync(h->stage_v[b], v, kb, cudaMemcpyHostToDevice, h->copy_stream)) != cudaSuccess ||
       (e = cudaMemcpyAsync(h->stage_pos[b], pos, pb, cudaMemcpyHostToDevice, h->copy_stream)) != cudaSuccess ||
       (e = cudaEventRecord(h->ev_h2d[b], h->copy_stream)) != cudaSuccess ||
-      (e = cudaStreamWaitEvent(cs, h->ev_h2d[b], 0)) != cudaSuccess)
+      (e = cudaStreamWaitEvent(cs, h->ev_h2d[b], 0)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(cs, h->ev_stage_free[b], 0)) != cudaSuccess)
     return set_err(h, STATEKV_ERR_CUDA, "host-to-device copy failed: %s", cudaGetErrorString(e));
   if (L->last_entry == 1) {
     // the layer's previous step came through the device-buffer call on the
