@@ -93,10 +93,12 @@ struct MergeArgs {
 // launch carries extra blocks that merge the attention's key-split partials
 // (not on the path to C_n).
 struct SelectArgs {
-  const float* part;      // part[s][g][j], j < m + T
+  const float* part;      // part[s][g * n_qsplit + q][j], j < m + T: the score pass's partial sums
   long long part_s;
-  int part_g;
-  float* pool_score;      // out, same layout as part (row of the selection group only)
+  int part_g;             // row stride of part and pool_score
+  int n_qsplit;           // rows of part per KV group
+  float* pool_score;      // out [s][g][j] (row of the selection group only)
+  long long pool_s;       // stream stride of pool_score
   const int32_t* pos_c;   // current C positions [s][g][B] (read in recency mode)
   const int32_t* pos_f;   // frame positions [s][T] (read in recency mode)
   int32_t* idx;           // out [s][g][B] kept pool indices, ascending (row 0 in global mode)

@@ -56,9 +56,10 @@ struct ScoreTcArgs {
   long long lse_s;
   const float* ml_part;  // [S][Hq][n_split][T] log2-sum-exp per key split (n_split > 1)
   int n_split;
-  float* part;       // [S][Hkv][pool]
+  float* part;       // [S][Hkv * n_qsplit][pool]: one row per (KV group, split of its query rows)
   long long part_s;
   int part_g;
+  int n_qsplit;      // splits of a group's query-row chunks over CTAs (>= 1)
   int m, T, Hq, Hkv, causal, n_c_tiles, n_f_tiles, S;
   float scale_log2;
   int* err;          // device error word (timeouts)
@@ -66,6 +67,10 @@ struct ScoreTcArgs {
 };
 cudaError_t launch_score_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kc, const CUtensorMap& tm_kf,
                             const ScoreTcArgs& a, int d, cudaStream_t st, bool pdl = false);
+// Splits of each group's query-row chunks for the score pass: enough CTAs to
+// cover n_sm when the key tiles alone do not, at most kMaxQsplit.
+constexpr int kMaxQsplit = 8;
+int score_tc_qsplit(int S, int Hq, int Hkv, int T, int m, int n_sm);
 
 // Tensor-core attention (bf16) over [compressed rows; frame tokens].
 // Query tiles: with stack = 0 a tile is 128 consecutive rows of one query

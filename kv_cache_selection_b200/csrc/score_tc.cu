@@ -20,6 +20,8 @@
 // while the MMA fills the fourth of the four TMEM accumulators.  Each
 // epilogue warp reads its lanes 16 columns at a time with the next TMEM load
 // in flight, and frees the accumulator as soon as its last load has landed.
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_common.cuh"
@@ -101,7 +103,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int s = blockIdx.z, g = blockIdx.y, tile = blockIdx.x;
+  // blockIdx.y = (KV group, split of the group's query-row chunks)
+  const int s = blockIdx.z, g = blockIdx.y / a.n_qsplit, qs = blockIdx.y % a.n_qsplit, tile = blockIdx.x;
   const bool is_c = tile < a.n_c_tiles;
   const int r0 = is_c ? tile * 128 : (tile - a.n_c_tiles) * 128;  // first C row / frame token
   const int G = a.Hq / a.Hkv;
@@ -110,7 +113,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ending before r0 hold nothing visible for this tile
   const int ic_min = (!is_c && a.causal) ? r0 / 128 : 0;
   const int per_head = n_ic - ic_min;
-  const int n_chunks = G * per_head;
+  // this CTA takes chunks [c_lo, c_lo + n_chunks) of the group's G * per_head
+  const int c_lo = qs * (G * per_head) / a.n_qsplit;
+  const int n_chunks = (qs + 1) * (G * per_head) / a.n_qsplit - c_lo;
 
   const uint32_t bar_k = sb + L::kBar;
   auto bar_qfull = [&](int st) { return sb + L::kBar + 8u * (1 + st); };
@@ -161,8 +166,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < n_chunks; ++c) {
         const int st = c % kStages;
         if (!mbar_wait(bar_qempty(st), ((c / kStages) & 1) ^ 1, a.err, kErrWaitEmpty, abort_flag, wait_lim)) break;
-        const int h = g * G + c / per_head;
-        const int i0 = (ic_min + c % per_head) * 128;
+        const int h = g * G + (c_lo + c) / per_head;
+        const int i0 = (ic_min + (c_lo + c) % per_head) * 128;
         mbar_arrive_expect_tx(bar_qfull(st), L::kTileBytes);
         for (int at = 0; at < L::kAtoms; ++at)
           tma_load_4d(sb + L::kQ + st * L::kTileBytes + at * L::kAtomBytes, &tm_q, bar_qfull(st), at * 64, h,
@@ -216,8 +221,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int bar_wg = 3 + half;                                            // named barrier of the warpgroup
     float mlv[8];
     auto load_stats = [&](int c) {
-      const int hh = c / per_head;
-      const int i = (ic_min + c % per_head) * 128 + r_wg;
+      const int hh = (c_lo + c) / per_head;
+      const int i = (ic_min + (c_lo + c) % per_head) * 128 + r_wg;
       const bool valid = i < a.T;
       const long long rowbase = (long long)(s * a.Hq + g * G + hh);
 #pragma unroll
@@ -246,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int c = half, it = 0; c < n_chunks; c += kGroups, ++it) {
       const int buf = c & 3;
-      const int i0 = (ic_min + c % per_head) * 128;
+      const int i0 = (ic_min + (c_lo + c) % per_head) * 128;
       float* lse2 = lse_wg + (it & 1) * 128;
       publish_stats(lse2);
       if (c + kGroups < n_chunks) load_stats(c + kGroups);
@@ -298,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool valid = is_c ? key < a.m : key < a.T;
       if (valid) {
         const int j = is_c ? key : a.m + key;
-        a.part[s * a.part_s + (long long)g * a.part_g + j] = tot;
+        a.part[s * a.part_s + (long long)(g * a.n_qsplit + qs) * a.part_g + j] = tot;
       }
     }
   }
@@ -312,11 +317,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
+int score_tc_qsplit(int S, int Hq, int Hkv, int T, int m, int n_sm) {
+  const int n_tiles = (m + 127) / 128 + (T + 127) / 128;
+  const int ctas = S * Hkv * n_tiles;
+  if (ctas <= 0 || Hkv <= 0) return 1;
+  const int chunks = (Hq / Hkv) * ((T + 127) / 128);  // query-row chunks of a group
+  int q = n_sm / ctas;
+  q = std::min(q, std::min(chunks, kMaxQsplit));
+  return std::max(q, 1);
+}
+
 cudaError_t launch_score_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kc, const CUtensorMap& tm_kf,
                             const ScoreTcArgs& a, int d, cudaStream_t st, bool pdl) {
   const int n_tiles = a.n_c_tiles + a.n_f_tiles;
   if (n_tiles == 0) return cudaSuccess;
-  dim3 grid(n_tiles, a.Hkv, a.S);
+  dim3 grid(n_tiles, a.Hkv * a.n_qsplit, a.S);
   cudaError_t e;
   if (d == 128) {
     const int smem = Smem<128>::kAlloc;

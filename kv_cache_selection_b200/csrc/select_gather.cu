@@ -107,7 +107,10 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
   // 1. scores of the pool: the KV groups' partial sums added in a fixed order
   //    (ascending group), written out as the pool scores and staged as bits
   const float* __restrict__ part = a.part + s * a.part_s;
-  float* pool_score = a.pool_score + s * a.part_s + (long long)G0 * a.part_g;
+  float* pool_score = a.pool_score + s * a.pool_s + (long long)G0 * a.part_g;
+  // rows of part summed for this group: the KV groups' (and within a group the
+  // query-row splits') partial sums, in ascending row order
+  const int R0 = G0 * a.n_qsplit, R1 = G1 * a.n_qsplit;
   uint32_t tmin = 0xffffffffu, tmax = 0u;  // span of this thread's staged values (first level)
   if ((a.part_g & 3) == 0 && (reinterpret_cast<uintptr_t>(part) & 15) == 0) {
     // four consecutive candidates per thread and group as one 16-byte load
@@ -116,12 +119,12 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
       const int j0 = 4 * c;
       const bool full = j0 + 3 < L;
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int gb = G0; gb < G1; gb += 8) {
+      for (int gb = R0; gb < R1; gb += 8) {
         float4 x[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           x[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (gb + u < G1) {
+          if (gb + u < R1) {
             const float* src = part + (long long)(gb + u) * a.part_g + j0;
             if (full) {
               x[u] = __ldg(reinterpret_cast<const float4*>(src));
@@ -167,7 +170,7 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
   } else {
     for (int j = threadIdx.x; j < L; j += kSelThreads) {
       float v = 0.f;
-      for (int g = G0; g < G1; ++g) v += __ldg(part + (long long)g * a.part_g + j);
+      for (int g = R0; g < R1; ++g) v += __ldg(part + (long long)g * a.part_g + j);
       pool_score[j] = v;
       if (!a.recency) {
         const uint32_t b = score_bits(v);

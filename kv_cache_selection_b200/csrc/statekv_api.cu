@@ -47,7 +47,7 @@ struct LayerState {
   // per-step scratch of this layer (each layer has its own, so that steps of
   // different layers may run concurrently on different streams)
   float* lse = nullptr;         // [S][Hq][T]
-  float* part = nullptr;        // [S][Hkv][B+T]
+  float* part = nullptr;        // [S][Hkv * query splits][B+T]
   float* pool_score = nullptr;  // [S][Hkv][B+T]
   int32_t* idx = nullptr;       // [S][Hkv][max(B,1)]
   __nv_bfloat16* o_part = nullptr;  // attention key-split partials (bf16 path)
@@ -169,7 +169,7 @@ int alloc_layer(statekv_t h, LayerState& L) {
   if ((rc = dev_alloc(h, (void**)&L.posd, (size_t)h->S * max_tok * 4))) return rc;
   const size_t S = h->S, pool = (size_t)h->B + h->T;
   if ((rc = dev_alloc(h, (void**)&L.lse, S * h->Hq * h->T * 4)) ||
-      (rc = dev_alloc(h, (void**)&L.part, S * h->Hkv * pool * 4)) ||
+      (rc = dev_alloc(h, (void**)&L.part, S * h->Hkv * skv::kMaxQsplit * pool * 4)) ||
       (rc = dev_alloc(h, (void**)&L.pool_score, S * h->Hkv * pool * 4)) ||
       (rc = dev_alloc(h, (void**)&L.idx, S * h->Hkv * std::max(h->B, 1) * 4)))
     return rc;
@@ -511,6 +511,7 @@ int prefill_step(statekv_t h, int layer, const void* q, const void* k, const voi
   }
 
   // (b) score pass
+  int n_qsplit = 1;  // rows of the partial-sum buffer per KV group
   skv::ScoreArgs sa{};
   sa.q = q;
   sa.q_s = aa.q_s;
@@ -539,8 +540,10 @@ int prefill_step(statekv_t h, int layer, const void* q, const void* k, const voi
     ta.lse_s = aa.lse_s;
     ta.ml_part = L->ml_part;
     ta.n_split = n_split;
+    ta.n_qsplit = skv::score_tc_qsplit(S, Hq, Hkv, T, m, h->n_sm);
+    n_qsplit = ta.n_qsplit;
     ta.part = L->part;
-    ta.part_s = sa.part_s;
+    ta.part_s = (long long)Hkv * n_qsplit * pool;
     ta.part_g = pool;
     ta.m = m;
     ta.T = T;
@@ -565,9 +568,11 @@ int prefill_step(statekv_t h, int layer, const void* q, const void* k, const voi
   // (c) top-B select
   skv::SelectArgs se{};
   se.part = L->part;
-  se.part_s = sa.part_s;
+  se.part_s = (long long)Hkv * n_qsplit * pool;
   se.part_g = pool;
+  se.n_qsplit = n_qsplit;
   se.pool_score = L->pool_score;
+  se.pool_s = (long long)Hkv * pool;
   se.pos_c = L->posc[cur];
   se.pos_f = pos;
   se.idx = L->idx;

@@ -195,7 +195,9 @@ extern "C" int statekv_step_noalloc(int Hq, int Hkv, int d, int T, int B, int dt
   se.part = part;
   se.part_s = sa.part_s;
   se.part_g = (int)pool;
+  se.n_qsplit = 1;
   se.pool_score = pool_score;
+  se.pool_s = sa.part_s;
   se.pos_c = posc;
   se.pos_f = pos;
   se.idx = idx;
