@@ -313,6 +313,19 @@ def test_8b_stack_layers_interleaved():
 
 
 @cuda
+@pytest.mark.parametrize("select", ["global", "per_kv_head"])
+def test_8b_shape_score_query_split(select):
+    """8B layer shape with B=2048 on one stream: the score pass splits each KV
+    group's query-row chunks over several CTAs (8 at frame 0, where only the
+    frame's two key tiles exist; 2 once C holds 2048 rows) and the selection
+    adds their partial-sum rows.  Checked while C fills and after it evicts,
+    in both selection modes."""
+    wl = Syn.workload("8b_layer", B=2048, frames=10)
+    r = run_stream_parity(wl, wl.frames, check={0, 1, 7, 8, 9}, select=select)
+    assert r["checked"] == 5
+
+
+@cuda
 def test_8b_sweep_shape_four_streams():
     """The sweep workload's launch shape: 4 streams per call at the 8B layer
     shape, with B=1024 so eviction starts at frame 4."""
