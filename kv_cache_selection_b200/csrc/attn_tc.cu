@@ -525,20 +525,40 @@ __global__ void __launch_bounds__(256) attn_merge_wide_kernel(AttnTcArgs a) {
   const long long sh = rw / a.T;  // s * Hq + h
   const int h = (int)(sh % a.Hq), s = (int)(sh / a.Hq);
   const long long prow0 = sh * a.n_split * a.T + i;
+  // eight splits' loads in flight per round (a decode has tens of splits)
+  constexpr int kB = 8;
   float mx = -INFINITY;
-  for (int u = 0; u < a.n_split; ++u) mx = fmaxf(mx, __ldg(a.ml_part + prow0 + (long long)u * a.T));
+  for (int u0 = 0; u0 < a.n_split; u0 += kB) {
+    float m8[kB];
+#pragma unroll
+    for (int k = 0; k < kB; ++k)
+      m8[k] = u0 + k < a.n_split ? __ldg(a.ml_part + prow0 + (long long)(u0 + k) * a.T) : -INFINITY;
+#pragma unroll
+    for (int k = 0; k < kB; ++k) mx = fmaxf(mx, m8[k]);
+  }
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float wsum = 0.f;
-  for (int u = 0; u < a.n_split; ++u) {
-    const float ml = __ldg(a.ml_part + prow0 + (long long)u * a.T);
-    if (ml == -INFINITY) continue;
-    const float w = ex2_approx(ml - mx);
-    const float4 o = __ldg(reinterpret_cast<const float4*>(a.o_part32 + (prow0 + (long long)u * a.T) * D) + chunk);
-    wsum += w;
-    acc.x += w * o.x;
-    acc.y += w * o.y;
-    acc.z += w * o.z;
-    acc.w += w * o.w;
+  for (int u0 = 0; u0 < a.n_split; u0 += kB) {
+    float m8[kB];
+    float4 o8[kB];
+#pragma unroll
+    for (int k = 0; k < kB; ++k) {
+      m8[k] = -INFINITY;
+      if (u0 + k < a.n_split) {
+        m8[k] = __ldg(a.ml_part + prow0 + (long long)(u0 + k) * a.T);
+        o8[k] = __ldg(reinterpret_cast<const float4*>(a.o_part32 + (prow0 + (long long)(u0 + k) * a.T) * D) + chunk);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kB; ++k) {
+      if (m8[k] == -INFINITY) continue;
+      const float w = ex2_approx(m8[k] - mx);
+      wsum += w;
+      acc.x += w * o8[k].x;
+      acc.y += w * o8[k].y;
+      acc.z += w * o8[k].z;
+      acc.w += w * o8[k].w;
+    }
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
   __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + s * a.out_s + (long long)i * a.out_row + (long long)h * D;
