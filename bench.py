@@ -554,8 +554,12 @@ def flatness_report(SKV, wl, dev):
 def decode_report(h, wl, dev, flush, n_texts=(1, 16, 64), reps=5):
     """Decode attention of n text tokens over the layer's whole detailed state
     (512 frames = 131,072 tokens): device time per call (CUDA events, L2
-    flushed before each call) against the HBM roofline; the algorithmic bytes
-    are D's K and V read once (2 * Hkv * N * d * 2) plus the text q, k, v, out."""
+    flushed before each call) against its roofline.  The algorithmic bytes
+    are D's K and V read once (2 * Hkv * N * d * 2) plus the text q, k, v, out;
+    the algorithmic FLOPs are 4 * Hq * d * (n * N + n (n + 1) / 2) (QK^T and
+    PV over D and the causal text block).  The bound is whichever of the two
+    takes longer at the peaks: HBM for a few text tokens, the tensor pipe once
+    G * n query rows share each K/V row (n = 64 at G = 7)."""
     peaks, src = load_peaks()
     N = h.frames(0) * wl.T
     res = {"workload": f"8b_layer: decode over D after {h.frames(0)} frames ({N} tokens)", "per_n_text": {}}
@@ -576,11 +580,20 @@ def decode_report(h, wl, dev, flush, n_texts=(1, 16, 64), reps=5):
         torch.cuda.synchronize()
         us = statistics.median(a.elapsed_time(b) for a, b in ts) * 1e3
         byts = 2 * wl.Hkv * N * wl.d * 2 + (2 * n * wl.Hq + 2 * n * wl.Hkv) * wl.d * 2
+        flops = 4 * wl.Hq * wl.d * (n * N + n * (n + 1) // 2)
         gbs = byts / us / 1e3
+        tflops = flops / us / 1e6
+        t_hbm = byts / (peaks["hbm_gbs"] * 1e3)       # us at the HBM peak
+        t_tc = flops / (peaks["bf16_tflops"] * 1e6)   # us at the bf16 tensor peak
         res["per_n_text"][n] = {"us": round(us, 2), "bytes": byts, "gbs": round(gbs, 1),
-                                "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+                                "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                                "flops": flops, "tflops": round(tflops, 1),
+                                "frac_of_tensor": round(tflops / peaks["bf16_tflops"], 4),
+                                "bound": "hbm" if t_hbm >= t_tc else "tensor",
+                                "frac": round(max(t_hbm, t_tc) / us, 4)}
     res["peak_gbs"] = peaks["hbm_gbs"]
-    res["peak_source"] = f"{src} (copy)"
+    res["peak_tflops"] = peaks["bf16_tflops"]
+    res["peak_source"] = f"{src} (copy; bf16 burst)"
     return res
 
 
