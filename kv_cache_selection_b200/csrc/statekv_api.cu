@@ -481,8 +481,8 @@ int prefill_step(statekv_t h, int layer, const void* q, const void* k, const voi
     ta.n_split = std::min(h->max_split, skv::attn_tc_splits(S, Hq, Hkv, T, m, h->n_sm));
     ta.nC = (m + 127) / 128;
     ta.nF = ta.n_it;
-  ta.stack = 0;
-  ta.q_rows = 128;
+    ta.stack = 0;
+    ta.q_rows = 128;
     ta.scale_log2 = scale_log2;
     ta.err = h->dev_err;
     ta.wait_ns = h->wait_ns;
