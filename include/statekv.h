@@ -193,15 +193,22 @@ typedef enum {
   STATEKV_STAGE_GATHER = 4,            /* (d) gather into C_n + append to D    */
   STATEKV_STAGE_DECODE = 5,            /* statekv_decode attention             */
   STATEKV_STAGE_DECODE_COMBINE = 6,    /* statekv_decode merge of key splits   */
+  STATEKV_STAGE_ATTENTION_CHAINED = 7, /* (a) attention and its split merge,   */
+                                       /*     one event pair (profiling mode 2) */
   STATEKV_N_STAGES = 8
 } statekv_stage;
 
-/* Per-stage device timing: when on, every later prefill_frame records a CUDA
+/* Per-stage device timing.  on = 1: every later prefill_frame records a CUDA
  * event pair around each kernel on the call's stream (a few microseconds of
  * extra enqueue cost; leave off in production), and the merge of the
  * attention's key splits, which otherwise rides in the select launch, runs as
  * its own launch so that its time is recorded under ATTENTION_COMBINE.
- * Turning it off drops unread records. */
+ * on = 2: the same, except that the attention and its merge share one event
+ * pair, recorded under ATTENTION_CHAINED, with the merge launched right behind
+ * the attention as a programmatic dependent launch (as the step chains its
+ * kernels), so that the pair times both kernels without a launch gap between
+ * them.  on = 0 turns timing off and drops unread records; any other value is
+ * STATEKV_ERR_INVALID_ARG. */
 int statekv_profile_enable(statekv_t h, int on);
 
 /* Accumulated device time and launch count per stage since the last read:

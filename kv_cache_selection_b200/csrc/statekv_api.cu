@@ -91,7 +91,7 @@ struct statekv_handle {
   std::vector<void*> allocs;
   // launch accounting and optional per-stage event timing
   long long launches = 0;
-  bool prof = false;
+  int prof = 0;  // 0 off, 1 per-kernel events, 2 attention and its merge as one stage
   struct Rec {
     int stage;
     cudaEvent_t a, b;
@@ -487,13 +487,19 @@ int prefill_step(statekv_t h, int layer, const void* q, const void* k, const voi
     ta.err = h->dev_err;
     ta.wait_ns = h->wait_ns;
     {
-      StageScope sc(h, st, STATEKV_STAGE_ATTENTION);
+      const bool chained = h->prof == 2 && ta.n_split > 1;
+      StageScope sc(h, st, chained ? STATEKV_STAGE_ATTENTION_CHAINED : STATEKV_STAGE_ATTENTION);
       if ((e = skv::launch_attn_tc(tq, tkc, tvc, tkf, tvf, ta, d, st, true)) != cudaSuccess)
         return launch_err(h, e, "attention");
+      if (chained) {
+        // profiling mode 2: the merge right behind the attention, in the same event pair
+        if ((e = skv::launch_attn_combine(ta, d, st, true)) != cudaSuccess) return launch_err(h, e, "attention merge");
+        ++h->launches;
+      }
       sc.done();
     }
     n_split = ta.n_split;
-    if (n_split > 1) {
+    if (n_split > 1 && h->prof != 2) {
       if (h->prof) {
         // timed runs charge the merge of the key splits to the attention stage
         // by launching it on its own; otherwise it rides in the select launch
@@ -885,6 +891,7 @@ int statekv_get_step_stats(statekv_t h, const float** lse, const float** pool_sc
 
 int statekv_profile_enable(statekv_t h, int on) {
   if (!h) return set_err(nullptr, STATEKV_ERR_INVALID_ARG, "null handle");
+  if (on < 0 || on > 2) return set_err(h, STATEKV_ERR_INVALID_ARG, "profiling mode %d (0, 1 or 2)", on);
   if (!on) {
     for (auto& r : h->recs) {
       h->ev_free.push_back(r.a);
@@ -892,7 +899,7 @@ int statekv_profile_enable(statekv_t h, int on) {
     }
     h->recs.clear();
   }
-  h->prof = on != 0;
+  h->prof = on;
   return STATEKV_OK;
 }
 

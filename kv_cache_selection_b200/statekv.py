@@ -21,7 +21,8 @@ BF16, F32 = 0, 1
 MASKS = {"frame_causal": 0, "frame_bidir": 1}
 SELECTS = {"global": 0, "per_kv_head": 1, "recency": 2}
 N_STAGES = 8
-STAGES = ["attention", "attention_combine", "score", "select", "gather", "decode", "decode_combine", None]
+STAGES = ["attention", "attention_combine", "score", "select", "gather", "decode", "decode_combine",
+          "attention_chained"]
 ERRORS = {0: "OK", -1: "INVALID_ARG", -2: "UNSUPPORTED", -3: "CAPACITY", -4: "OOM", -5: "CUDA"}
 
 if not os.path.exists(LIB_PATH):
@@ -167,7 +168,10 @@ class StateKV:
         _check(rc, self._h)
         return out
 
-    def profile(self, on: bool = True):
+    def profile(self, on=True):
+        """Per-stage device timing: False/0 off, True/1 one event pair per
+        kernel, 2 the attention and its split merge under one event pair
+        (stage "attention_chained")."""
         _check(lib.statekv_profile_enable(self._h, int(on)), self._h)
 
     def profile_read(self):

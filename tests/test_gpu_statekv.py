@@ -703,3 +703,45 @@ def test_layers_pipelined_on_two_streams_match_in_order():
     assert h.device_status() == 0
     h.close()
     ref.close()
+
+
+@cuda
+def test_profiling_modes_time_the_same_step():
+    """Per-stage timing changes how the step is launched (mode 1: the split
+    merge on its own, events around every kernel; mode 2: the attention and
+    its merge under one event pair) but not what it computes: every mode
+    gives bit-identical out, C and D, and records the expected stages."""
+    S = _skv()
+    wl = Syn.workload("1b_layer")
+    dev = torch.device("cuda")
+    n_frames = 7            # C fills after 4 frames (B = 1024, T = 256): 3 steady-state steps
+    frames = [tuple(t.to(dev) for t in Syn.gen_frame(wl, n)) for n in range(n_frames)]
+    results = {}
+    for mode in (0, 1, 2):
+        h = S.StateKV(wl.Hq, wl.Hkv, wl.d, wl.T, wl.B, max_frames=n_frames, dtype=wl.dtype)
+        h.profile(mode)
+        outs = [h.prefill_frame(0, *f).clone() for f in frames]
+        torch.cuda.synchronize()
+        rec = h.profile_read() if mode else {}
+        C, D = h.get_compressed(0), h.get_detailed(0)
+        results[mode] = (outs, {k: v.clone() for k, v in C.items() if isinstance(v, torch.Tensor)},
+                         {k: v.clone() for k, v in D.items() if isinstance(v, torch.Tensor)})
+        if mode == 1:
+            for st in ("attention", "attention_combine", "score", "select", "gather"):
+                assert rec[st][1] == n_frames, (st, rec[st])
+            assert rec["attention_chained"][1] == 0
+        if mode == 2:
+            assert rec["attention_chained"][1] == n_frames
+            assert rec["attention_combine"][1] == 0 and rec["attention"][1] == 0
+            assert all(rec[st][1] == n_frames for st in ("score", "select", "gather"))
+            assert rec["attention_chained"][0] > 0.0
+        with pytest.raises(S.StateKVError):
+            h.profile(3)
+        assert h.device_status() == 0
+        h.close()
+    for mode in (1, 2):
+        for a, b in zip(results[0][0], results[mode][0]):
+            assert torch.equal(a, b)
+        for part in (1, 2):
+            for key, t in results[0][part].items():
+                assert torch.equal(t, results[mode][part][key]), (mode, key)
