@@ -572,7 +572,7 @@ def flatness_report(SKV, wl, dev):
     return rep, dec
 
 
-def decode_report(h, wl, dev, flush, n_texts=(1, 16, 64), reps=5):
+def decode_report(h, wl, dev, flush, n_texts=(1, 16, 64), reps=20):
     """Decode attention of n text tokens over the layer's whole detailed state
     (512 frames = 131,072 tokens): device time per call (CUDA events, L2
     flushed before each call) against its roofline.  The algorithmic bytes
@@ -599,7 +599,9 @@ def decode_report(h, wl, dev, flush, n_texts=(1, 16, 64), reps=5):
             e1.record()
             ts.append((e0, e1))
         torch.cuda.synchronize()
-        us = statistics.median(a.elapsed_time(b) for a, b in ts) * 1e3
+        # the mean of the calls: single event intervals come in steps of ~2 us
+        # on this part, which a median of a few calls would keep
+        us = statistics.fmean(a.elapsed_time(b) for a, b in ts) * 1e3
         byts = 2 * wl.Hkv * N * wl.d * 2 + (2 * n * wl.Hq + 2 * n * wl.Hkv) * wl.d * 2
         flops = 4 * wl.Hq * wl.d * (n * N + n * (n + 1) // 2)
         gbs = byts / us / 1e3

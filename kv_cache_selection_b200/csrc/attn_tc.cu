@@ -508,9 +508,10 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(MergeArgs a) {
   merge_chunk<D>(a, (long long)blockIdx.x * blockDim.x + threadIdx.x);
 }
 
-// Merge of n_split float32 partials (O/l and log2-sum-exp per split): thread
-// = (row, 4-element chunk of d); pass 1 takes the largest log2-sum-exp, pass
-// 2 adds the splits' O/l weighted by 2^(ml_u - max).
+// Merge of n_split float32 partials (O/l and log2-sum-exp per split) when the
+// rows alone fill the GPU: thread = (row, 4-element chunk of d); pass 1 takes
+// the largest log2-sum-exp, pass 2 adds the splits' O/l weighted by
+// 2^(ml_u - max).
 template <int D>
 __global__ void __launch_bounds__(256) attn_merge_wide_kernel(AttnTcArgs a) {
   pdl_wait();
@@ -570,13 +571,118 @@ __global__ void __launch_bounds__(256) attn_merge_wide_kernel(AttnTcArgs a) {
     a.lse[s * a.lse_s + (long long)h * a.T + i] = wsum > 0.f ? (mx + __log2f(wsum)) * kLn2 : -INFINITY;
 }
 
+// The same merge when the rows are few (a decode of a few text tokens has
+// tens of splits per row): one block per query row, so that the work still
+// spreads over many threads with every load of a pass in flight at once:
+//   1. each thread takes a split's log2-sum-exp ml_u; block maximum mx;
+//   2. w_u = 2^(ml_u - mx) into shared memory, wsum = sum of the w_u (a fixed
+//      reduction tree);
+//   3. thread (group g, 4-element chunk c) adds w_u * (O/l)_u[c] over the
+//      splits u = g, g + kG, ...; the kG group sums are added in group order.
+// out = sum / wsum; lse = mx + log2(wsum), in natural-log units.
+template <int D>
+__global__ void __launch_bounds__(256) attn_merge_split_kernel(AttnTcArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  constexpr int kT = 256;
+  constexpr int kChunks = D / 4;       // 4-float chunks of a row
+  constexpr int kG = kT / kChunks;     // split groups
+  constexpr int kBatch = 8;            // loads in flight per thread and round
+  __shared__ float s_w[kMaxMergeSplit];
+  __shared__ float s_red[kT / 32];
+  __shared__ float4 s_acc[kG][kChunks];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const long long rw = blockIdx.x;     // (s, h, i)
+  const int i = (int)(rw % a.T);
+  const long long sh = rw / a.T;       // s * Hq + h
+  const int h = (int)(sh % a.Hq), s = (int)(sh / a.Hq);
+  const long long prow0 = sh * a.n_split * a.T + i;
+  const int n = a.n_split;
+  // 1. largest log2-sum-exp of the row
+  float mx = -INFINITY;
+  for (int u = tid; u < n; u += kT) mx = fmaxf(mx, __ldg(a.ml_part + prow0 + (long long)u * a.T));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  if (lane == 0) s_red[warp] = mx;
+  __syncthreads();
+  mx = s_red[0];
+#pragma unroll
+  for (int w = 1; w < kT / 32; ++w) mx = fmaxf(mx, s_red[w]);
+  __syncthreads();  // s_red is reused below
+  // 2. split weights (0 for a split that saw no key of the row)
+  float wpart = 0.f;
+  for (int u = tid; u < n; u += kT) {
+    const float ml = __ldg(a.ml_part + prow0 + (long long)u * a.T);
+    const float w = ml == -INFINITY ? 0.f : ex2_approx(ml - mx);
+    s_w[u] = w;
+    wpart += w;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) wpart += __shfl_xor_sync(0xffffffffu, wpart, off);
+  if (lane == 0) s_red[warp] = wpart;
+  __syncthreads();
+  float wsum = 0.f;
+#pragma unroll
+  for (int w = 0; w < kT / 32; ++w) wsum += s_red[w];
+  // 3. weighted sum of the splits' O/l, kBatch loads in flight per round
+  const int c = tid % kChunks, g = tid / kChunks;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int u0 = g; u0 < n; u0 += kG * kBatch) {
+    float4 o[kBatch];
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) {
+      const int u = u0 + k * kG;
+      if (u < n) o[k] = __ldg(reinterpret_cast<const float4*>(a.o_part32 + (prow0 + (long long)u * a.T) * D) + c);
+    }
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) {
+      const int u = u0 + k * kG;
+      if (u < n) {
+        const float w = s_w[u];
+        acc.x += w * o[k].x;
+        acc.y += w * o[k].y;
+        acc.z += w * o[k].z;
+        acc.w += w * o[k].w;
+      }
+    }
+  }
+  s_acc[g][c] = acc;
+  __syncthreads();
+  if (g == 0) {
+#pragma unroll
+    for (int gg = 1; gg < kG; ++gg) {
+      const float4 x = s_acc[gg][c];
+      acc.x += x.x;
+      acc.y += x.y;
+      acc.z += x.z;
+      acc.w += x.w;
+    }
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+    __nv_bfloat16* orow =
+        static_cast<__nv_bfloat16*>(a.out) + s * a.out_s + (long long)i * a.out_row + (long long)h * D;
+    uint2 pk;
+    pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+    pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    reinterpret_cast<uint2*>(orow)[c] = pk;
+    if (c == 0 && a.lse)
+      a.lse[s * a.lse_s + (long long)h * a.T + i] = wsum > 0.f ? (mx + __log2f(wsum)) * kLn2 : -INFINITY;
+  }
+}
+
 }  // namespace
 
-cudaError_t launch_attn_merge_wide(const AttnTcArgs& a, int d, cudaStream_t st, bool pdl) {
+cudaError_t launch_attn_merge_wide(const AttnTcArgs& a, int d, int n_sm, cudaStream_t st, bool pdl) {
   const long long rows = (long long)a.S * a.Hq * a.T;
-  const int blocks = (int)((rows * (d / 4) + 255) / 256);
-  if (d == 128) return launch_kernel(attn_merge_wide_kernel<128>, dim3(blocks), dim3(256), 0, st, pdl, a);
-  return launch_kernel(attn_merge_wide_kernel<64>, dim3(blocks), dim3(256), 0, st, pdl, a);
+  if (a.n_split > kMaxMergeSplit) return cudaErrorInvalidValue;
+  const long long threads = rows * (d / 4);  // one thread per (row, 4-element chunk)
+  if (threads >= (long long)n_sm * 256) {
+    // the rows fill every SM with a block or more
+    const int blocks = (int)((threads + 255) / 256);
+    if (d == 128) return launch_kernel(attn_merge_wide_kernel<128>, dim3(blocks), dim3(256), 0, st, pdl, a);
+    return launch_kernel(attn_merge_wide_kernel<64>, dim3(blocks), dim3(256), 0, st, pdl, a);
+  }
+  if (d == 128) return launch_kernel(attn_merge_split_kernel<128>, dim3((unsigned)rows), dim3(256), 0, st, pdl, a);
+  return launch_kernel(attn_merge_split_kernel<64>, dim3((unsigned)rows), dim3(256), 0, st, pdl, a);
 }
 
 int attn_tc_splits(int S, int Hq, int Hkv, int T, int m, int n_sm) {

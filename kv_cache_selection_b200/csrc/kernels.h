@@ -35,6 +35,10 @@ cudaError_t ensure_dynamic_smem(void (*kernel)(KArgs...), int bytes) {
   return ensure_dynamic_smem(reinterpret_cast<const void*>(kernel), bytes);
 }
 
+// Most key splits the float32 merge of a decode takes (its weights sit in
+// shared memory).
+constexpr int kMaxMergeSplit = 256;
+
 constexpr int kDtypeBF16 = 0;
 constexpr int kDtypeF32 = 1;
 
@@ -100,8 +104,10 @@ cudaError_t launch_attn_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kc, co
                            const CUtensorMap& tm_kf, const CUtensorMap& tm_vf, const AttnTcArgs& a, int d,
                            cudaStream_t st, bool pdl = false);
 cudaError_t launch_attn_combine(const AttnTcArgs& a, int d, cudaStream_t st, bool pdl = false);
-// Merge of any number of float32 key-split partials (o_part32) into out and lse.
-cudaError_t launch_attn_merge_wide(const AttnTcArgs& a, int d, cudaStream_t st, bool pdl = false);
+// Merge of up to kMaxMergeSplit float32 key-split partials (o_part32) into out
+// and lse: thread-per-(row, chunk) when the rows fill the n_sm SMs, else one
+// block per row.
+cudaError_t launch_attn_merge_wide(const AttnTcArgs& a, int d, int n_sm, cudaStream_t st, bool pdl = false);
 MergeArgs merge_args(const AttnTcArgs& a, int d);
 
 // Message for statekv_last_error(NULL) (errors of calls without a handle).

@@ -796,7 +796,7 @@ int statekv_decode(statekv_t h, int layer, const void* q, const void* k, const v
   ta.wait_ns = h->wait_ns;
   const int units = S * Hkv * ta.n_pairs;
   int split = std::max(1, h->n_sm / std::max(units, 1));
-  split = std::min(split, std::min(ta.nC + ta.nF, 256));
+  split = std::min(split, std::min(ta.nC + ta.nF, skv::kMaxMergeSplit));
   ta.n_split = split;
   if (split > 1) {
     const size_t ob = (size_t)S * Hq * split * n_text * d * 4, mb = (size_t)S * Hq * split * n_text * 4;
@@ -846,7 +846,7 @@ int statekv_decode(statekv_t h, int layer, const void* q, const void* k, const v
   }
   if (split > 1) {
     StageScope sc(h, st, STATEKV_STAGE_DECODE_COMBINE);
-    if ((e = skv::launch_attn_merge_wide(ta, d, st, true)) != cudaSuccess) return launch_err(h, e, "decode merge");
+    if ((e = skv::launch_attn_merge_wide(ta, d, h->n_sm, st, true)) != cudaSuccess) return launch_err(h, e, "decode merge");
     sc.done();
   }
   return STATEKV_OK;
