@@ -675,8 +675,8 @@ cudaError_t launch_attn_merge_wide(const AttnTcArgs& a, int d, int n_sm, cudaStr
   const long long rows = (long long)a.S * a.Hq * a.T;
   if (a.n_split > kMaxMergeSplit) return cudaErrorInvalidValue;
   const long long threads = rows * (d / 4);  // one thread per (row, 4-element chunk)
-  if (threads >= (long long)n_sm * 256) {
-    // the rows fill every SM with a block or more
+  if (threads >= (long long)n_sm * 32) {
+    // a warp or more per SM: the rows give enough parallel loads
     const int blocks = (int)((threads + 255) / 256);
     if (d == 128) return launch_kernel(attn_merge_wide_kernel<128>, dim3(blocks), dim3(256), 0, st, pdl, a);
     return launch_kernel(attn_merge_wide_kernel<64>, dim3(blocks), dim3(256), 0, st, pdl, a);

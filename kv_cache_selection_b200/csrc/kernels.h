@@ -105,8 +105,8 @@ cudaError_t launch_attn_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_kc, co
                            cudaStream_t st, bool pdl = false);
 cudaError_t launch_attn_combine(const AttnTcArgs& a, int d, cudaStream_t st, bool pdl = false);
 // Merge of up to kMaxMergeSplit float32 key-split partials (o_part32) into out
-// and lse: thread-per-(row, chunk) when the rows fill the n_sm SMs, else one
-// block per row.
+// and lse: thread-per-(row, chunk) when that gives a warp or more per SM (of
+// n_sm), else one block per row.
 cudaError_t launch_attn_merge_wide(const AttnTcArgs& a, int d, int n_sm, cudaStream_t st, bool pdl = false);
 MergeArgs merge_args(const AttnTcArgs& a, int d);
 
