@@ -89,8 +89,14 @@ def _torch_dtype(code: int):
     return torch.bfloat16 if code == BF16 else torch.float32
 
 
-def _stream_ptr(stream) -> int:
+# the current stream's handle without building a torch.cuda.Stream object
+_raw_current_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
+def _stream_ptr(stream, device_index=None) -> int:
     if stream is None:
+        if _raw_current_stream is not None and device_index is not None:
+            return _raw_current_stream(device_index)
         stream = torch.cuda.current_stream()
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
@@ -117,9 +123,9 @@ def borrow(ptr: int, shape, dtype: torch.dtype) -> torch.Tensor:
 def _need(t: torch.Tensor, shape, dtype, name):
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch tensor")
-    if t.device.type != "cuda":
+    if not t.is_cuda:
         raise ValueError(f"{name} must be on a CUDA device")
-    if tuple(t.shape) != tuple(shape):
+    if t.shape != shape:
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
     if t.dtype != dtype:
         raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
@@ -137,6 +143,8 @@ class StateKV:
         self.dtype_code = _dtype_code(dtype)
         self.dtype = _torch_dtype(self.dtype_code)
         self.mask, self.select = mask, select
+        lead = () if n_streams == 1 else (n_streams,)
+        self._step_shapes = (lead + (T, Hq, d), lead + (T, Hkv, d), lead + (T,))  # q/out, k/v, pos
         h = ctypes.c_void_p()
         rc = lib.statekv_create_batched(ctypes.byref(h), n_streams, Hq, Hkv, d, T, B, max_frames,
                                         self.dtype_code, MASKS[mask], SELECTS[select])
@@ -155,16 +163,16 @@ class StateKV:
 
     def prefill_frame(self, layer, q, k, v, pos, out=None, stream=None):
         """One cache-builder step; returns out [.., T, Hq, d]."""
-        L = self._lead()
-        _need(q, L + (self.T, self.Hq, self.d), self.dtype, "q")
-        _need(k, L + (self.T, self.Hkv, self.d), self.dtype, "k")
-        _need(v, L + (self.T, self.Hkv, self.d), self.dtype, "v")
-        _need(pos, L + (self.T,), torch.int32, "pos")
+        sq, skv, sp = self._step_shapes
+        _need(q, sq, self.dtype, "q")
+        _need(k, skv, self.dtype, "k")
+        _need(v, skv, self.dtype, "v")
+        _need(pos, sp, torch.int32, "pos")
         if out is None:
             out = torch.empty_like(q)
-        _need(out, L + (self.T, self.Hq, self.d), self.dtype, "out")
+        _need(out, sq, self.dtype, "out")
         rc = lib.statekv_prefill_frame(self._h, layer, q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                       pos.data_ptr(), out.data_ptr(), _stream_ptr(stream))
+                                       pos.data_ptr(), out.data_ptr(), _stream_ptr(stream, q.get_device()))
         _check(rc, self._h)
         return out
 
