@@ -897,7 +897,7 @@ def main(argv=None):
     ap.add_argument("--mode", choices=["headline", "flatness", "stack", "sweep", "diagnostics"], default="headline",
                     help="headline: the contract's JSON line; others: report lines")
     ap.add_argument("--stack-frames", type=int, default=0)
-    ap.add_argument("--stack-pipeline", type=int, default=2, help="streams of the pipelined stack schedule")
+    ap.add_argument("--stack-pipeline", type=int, default=4, help="streams of the pipelined stack schedule")
     ap.add_argument("--diag-frames", type=int, default=64)
     ap.add_argument("--diag-b", type=int, default=1024, help="budget of the retained sets compared")
     ap.add_argument("--diag-budgets", type=int, nargs="+", default=[1, 16, 256, 1024, 4096])
