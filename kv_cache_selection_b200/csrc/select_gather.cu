@@ -115,35 +115,29 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
   if ((a.part_g & 3) == 0 && (reinterpret_cast<uintptr_t>(part) & 15) == 0) {
     // four consecutive candidates per thread and group as one 16-byte load
     const int n4 = (L + 3) / 4;
-    for (int c = threadIdx.x; c < n4; c += kSelThreads) {
-      const int j0 = 4 * c;
-      const bool full = j0 + 3 < L;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int gb = R0; gb < R1; gb += 8) {
-        float4 x[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          x[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (gb + u < R1) {
-            const float* src = part + (long long)(gb + u) * a.part_g + j0;
-            if (full) {
-              x[u] = __ldg(reinterpret_cast<const float4*>(src));
-            } else {
-              x[u].x = __ldg(src);
-              if (j0 + 1 < L) x[u].y = __ldg(src + 1);
-              if (j0 + 2 < L) x[u].z = __ldg(src + 2);
-            }
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          v.x += x[u].x;
-          v.y += x[u].y;
-          v.z += x[u].z;
-          v.w += x[u].w;
+    // one row's four candidates at j0 (zeros past the pool or past row R1)
+    auto load4 = [&](int j0, int row, float4& x) {
+      x = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (row < R1 && j0 < L) {
+        const float* src = part + (long long)row * a.part_g + j0;
+        if (j0 + 3 < L) {
+          x = __ldg(reinterpret_cast<const float4*>(src));
+        } else {
+          x.x = __ldg(src);
+          if (j0 + 1 < L) x.y = __ldg(src + 1);
+          if (j0 + 2 < L) x.z = __ldg(src + 2);
         }
       }
-      if (full && (reinterpret_cast<uintptr_t>(pool_score) & 15) == 0) {
+    };
+    auto add4 = [](float4& v, const float4& x) {
+      v.x += x.x;
+      v.y += x.y;
+      v.z += x.z;
+      v.w += x.w;
+    };
+    // the four candidates' scores out, their bits staged, the span updated
+    auto finish = [&](int j0, const float4& v) {
+      if (j0 + 3 < L && (reinterpret_cast<uintptr_t>(pool_score) & 15) == 0) {
         *reinterpret_cast<float4*>(pool_score + j0) = v;
         if (!a.recency) {
           const uint4 b4 = make_uint4(score_bits(v.x), score_bits(v.y), score_bits(v.z), score_bits(v.w));
@@ -165,6 +159,40 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
             }
           }
         }
+      }
+    };
+    if (R1 - R0 <= 4) {
+      // at most four rows: two columns per thread, all eight loads in one
+      // round (rows added in ascending order, as below)
+      for (int c = threadIdx.x; c < n4; c += 2 * kSelThreads) {
+        const int c1 = c + kSelThreads;
+        float4 x[8];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          load4(4 * c, R0 + u, x[u]);
+          load4(4 * c1, R0 + u, x[4 + u]);
+        }
+        float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          add4(v0, x[u]);
+          add4(v1, x[4 + u]);
+        }
+        finish(4 * c, v0);
+        if (c1 < n4) finish(4 * c1, v1);
+      }
+    } else {
+      for (int c = threadIdx.x; c < n4; c += kSelThreads) {
+        const int j0 = 4 * c;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int gb = R0; gb < R1; gb += 8) {
+          float4 x[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) load4(j0, gb + u, x[u]);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) add4(v, x[u]);
+        }
+        finish(j0, v);
       }
     }
   } else {
