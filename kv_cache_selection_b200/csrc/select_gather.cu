@@ -62,9 +62,10 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* w
 // B-th largest value) is found by histogram refinement: the values still in
 // play span [umin, umax]; a 4096-bin histogram over that span (bin width
 // 2^shift) locates the bin holding the B-th largest; the bin becomes the new
-// span.  As soon as that bin is one value wide (tau found) or holds at most 32
-// candidates, the refinement stops and one warp ranks those candidates
-// exactly by (value desc, pool index asc).  The result is (tau, need_eq): keep
+// span.  As soon as that bin is one value wide (tau found), is kept whole
+// (tau just below it), or holds at most 32 candidates, the refinement stops;
+// in the last case one warp ranks those candidates exactly by (value desc,
+// pool index asc).  The result is (tau, need_eq): keep
 // every candidate above tau and the first need_eq candidates equal to tau in
 // pool order, which is position order, so ties go to the lower position.
 constexpr int kBins = 4096;
@@ -336,6 +337,13 @@ __global__ void __launch_bounds__(kSelThreads) select_topb_kernel(SelectArgs a) 
       if (shift == 0) {  // the bin is one value
         tau = lo;
         need_eq = need;
+        break;
+      }
+      if (in_bin == need && lo > 0u) {
+        // every candidate of the bin is kept: the kept set is every value
+        // >= lo, with no tie to break (equal values share a bin)
+        tau = lo - 1u;
+        need_eq = 0u;
         break;
       }
       if (in_bin <= 32u) {
