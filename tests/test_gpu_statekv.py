@@ -565,9 +565,12 @@ def test_decode_other_groups(d, Hq, Hkv):
 
 
 @cuda
-def test_decode_batched_streams():
+@pytest.mark.parametrize("n_text", [1, 12])
+def test_decode_batched_streams(n_text):
+    """Three streams; one text token takes the block-per-row merge of the
+    split partials, twelve the row-parallel one."""
     wl = Syn.workload("1b_layer", Hq=14, Hkv=2, d=64, T=64, B=192)
-    _decode_case(wl, 6, 12, "bf16", n_streams=3)
+    _decode_case(wl, 6, n_text, "bf16", n_streams=3)
 
 
 @cuda
