@@ -50,13 +50,27 @@ def rank_info():
             int(os.environ.get("WORLD_SIZE", 1)))
 
 
-def load_peaks():
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+def load_peaks(path=None):
+    """Roofline denominators: the measured peaks file when it gives them
+    (positive numbers under the fallback's keys), else the fallback figures;
+    the second value says which ("measured", "measured+fallback" when the
+    file gives only some of them, or "fallback")."""
+    p = path or os.path.join(ROOT, "MEASURED_PEAKS.json")
+    peaks, found = dict(FALLBACK_PEAKS), 0
     if os.path.exists(p):
-        with open(p) as f:
-            d = json.load(f)
-        return d, "measured"
-    return dict(FALLBACK_PEAKS), "fallback"
+        try:
+            with open(p) as f:
+                d = json.load(f)
+        except (OSError, ValueError):
+            d = {}
+        for k in FALLBACK_PEAKS:
+            v = d.get(k) if isinstance(d, dict) else None
+            if isinstance(v, (int, float)) and not isinstance(v, bool) and v > 0:
+                peaks[k] = float(v)
+                found += 1
+    if found == len(FALLBACK_PEAKS):
+        return peaks, "measured"
+    return peaks, ("measured+fallback" if found else "fallback")
 
 
 def step_work(wl, m, S=1, causal=True):

@@ -92,3 +92,27 @@ def test_reference_arm_prints_the_contract_line(monkeypatch, capsys):
     assert d["value"] > 0 and d["steps"] == 1 and d["warmup"] == 3
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_peaks_file_read_with_fallback_for_missing_keys(tmp_path):
+    """The measured peaks are used when present; missing, malformed or
+    non-positive entries fall back to the stated fallback figures."""
+    import json
+    sys.path.insert(0, ROOT)
+    import bench
+    full = tmp_path / "full.json"
+    full.write_text(json.dumps({"hbm_gbs": 6541.0, "bf16_tflops": 1654.5, "bf16_tflops_sustained": 1420.0,
+                                "clocks": {"sm_mhz": 1965}}))
+    peaks, src = bench.load_peaks(str(full))
+    assert src == "measured" and peaks["bf16_tflops"] == 1654.5 and peaks["hbm_gbs"] == 6541.0
+    part = tmp_path / "part.json"
+    part.write_text(json.dumps({"hbm_gbs": 6541.0, "bf16_tflops": "n/a"}))
+    peaks, src = bench.load_peaks(str(part))
+    assert src == "measured+fallback" and peaks["hbm_gbs"] == 6541.0
+    assert peaks["bf16_tflops"] == bench.FALLBACK_PEAKS["bf16_tflops"]
+    bad = tmp_path / "bad.json"
+    bad.write_text("{not json")
+    peaks, src = bench.load_peaks(str(bad))
+    assert src == "fallback" and peaks == bench.FALLBACK_PEAKS
+    peaks, src = bench.load_peaks(str(tmp_path / "absent.json"))
+    assert src == "fallback" and peaks == bench.FALLBACK_PEAKS
